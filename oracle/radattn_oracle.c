@@ -1,0 +1,297 @@
+/*
+ * radattn_oracle.c -- plain CPU oracle for static-mask sparse attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only tests/, the smoke check in __graft_entry__.py and the
+ * cpu_baseline / reference arm of bench.py use it.  It shares no code, header,
+ * table or constant generator with the CUDA library; it restates the method
+ * from its published definition, slowly and in the most direct order.
+ *
+ * Sources followed (page title, then section / equation):
+ *   [RA]  "Radial Attention: O(n log n) Sparse Attention with Energy Decay for
+ *         Long Video Generation" (summary page):
+ *           eq. 1  dense attention softmax(QK^T/sqrt(d))V
+ *           eq. 2  sparse attention softmax((QK^T + M)/sqrt(d))V, M in {-inf,0}
+ *           eq. 3  token index j*s + l (frame j, in-frame position l)
+ *           eq. 4  the 4D radial mask M~[i,j,k,l]
+ *           eq. 5-6 zero-count bound (checked by the tests, not here)
+ *           sec. 6 "128x128 block-level sparsity granularity"
+ *   [TR]  "Token Radius Attention" tutorial with code, sec. 3.1 (tokens are
+ *         (t h w) flattened), sec. 3.2 / 4.2 / 5 (cube neighbourhood of
+ *         temporal radius r_t and spatial radius r_s)
+ *   [VR]  "Vera 1.1" temporal module, sec. 2.1-2.2 (causal AND sliding window:
+ *         query frame i sees key frames [max(0, i-W+1), i])
+ *
+ * Readings taken where the pages are silent or ambiguous:
+ *   - floor(log2(x)) is evaluated exactly as (bit length of x) - 1.
+ *   - |k-l| is the distance of in-frame flattened positions (eq. 3, eq. 4).
+ *   - the condition |k-l|+1 <= s / 2^b is a real-number comparison, tested
+ *     exactly as (|k-l|+1) * 2^b <= s.
+ *   - a 128x128 tile is kept iff at least one valid (query, key) pair in it is
+ *     kept; FULL iff all 128*128 pairs are valid and kept; otherwise PARTIAL.
+ *   - the 3D window excludes out-of-grid neighbours (no zero padding) and uses
+ *     softmax over the neighbour set, as the tutorial's own note asks.
+ *   - the sliding window keeps key frames with 0 <= i - j <= W - 1 (the prose
+ *     interval; the printed pseudocode has an off-by-one and a typo).
+ *   - a query row with no kept key outputs 0 with log-sum-exp -inf.
+ *
+ * All floating point is fp64; bf16 inputs are widened exactly.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* mask families and modes: same numeric values as the library's public enums,
+ * restated here so the two sides share no header. */
+#define OR_DENSE 0
+#define OR_RADIAL 1
+#define OR_WINDOW3D 2
+#define OR_SWC 3
+
+#define OR_TOKEN_EXACT 0
+#define OR_BLOCK 1
+
+#define OR_TILE_PARTIAL 0
+#define OR_TILE_FULL 1
+
+#define OR_TILE 128 /* [RA] sec. 6: 128x128 block granularity */
+
+#define OR_IN_BF16 0
+#define OR_IN_F32 1
+#define OR_IN_F64 2
+
+typedef struct {
+    int family;
+    int f;             /* frames */
+    int s;             /* tokens per frame */
+    int grid_h;        /* 3D window: s == grid_h * grid_w */
+    int grid_w;
+    int r_t;           /* 3D window: temporal radius */
+    int r_s;           /* 3D window: spatial radius */
+    int window_frames; /* sliding window: W */
+} or_spec;
+
+/* Threads the parallel loops below use. */
+int oracle_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+static long long or_abs(long long x) { return x < 0 ? -x : x; }
+
+/* floor(log2(x)) for x >= 1: position of the highest set bit. */
+static int or_floor_log2(long long x)
+{
+    int b = -1;
+    while (x > 0) {
+        x >>= 1;
+        b++;
+    }
+    return b;
+}
+
+/* [RA] eq. 4 for query (frame i, position k) and key (frame j, position l). */
+static int or_radial_kept(long long i, long long j, long long k, long long l, long long s)
+{
+    long long dist = or_abs(i - j);
+    long long w = 1LL << or_floor_log2(dist > 1 ? dist : 1); /* 2^floor(log2(max(|i-j|,1))) */
+    /* first case: w <= s and |k-l| + 1 <= s / w */
+    if (w <= s && (or_abs(k - l) + 1) * w <= s)
+        return 1;
+    /* second case: |i-j| mod ceil(w / s) == 0 and k == l */
+    long long period = (w + s - 1) / s;
+    if (dist % period == 0 && k == l)
+        return 1;
+    return 0;
+}
+
+/* [TR] sec. 3.2 / 4.2: the (2 r_t + 1) x (2 r_s + 1)^2 cube around the query. */
+static int or_window3d_kept(const or_spec* sp, long long q, long long key)
+{
+    long long s = sp->s, gw = sp->grid_w;
+    long long tq = q / s, pq = q % s, tk = key / s, pk = key % s;
+    long long hq = pq / gw, wq = pq % gw, hk = pk / gw, wk = pk % gw;
+    return or_abs(tq - tk) <= sp->r_t && or_abs(hq - hk) <= sp->r_s && or_abs(wq - wk) <= sp->r_s;
+}
+
+/* [VR] sec. 2.2: causal and at most W frames back, own frame included. */
+static int or_swc_kept(const or_spec* sp, long long q, long long key)
+{
+    long long i = q / sp->s, j = key / sp->s;
+    return (i - j) >= 0 && (i - j) <= (long long)sp->window_frames - 1;
+}
+
+/* M[q, key] == 0 ?  (token index = frame * s + position, [RA] eq. 3) */
+int oracle_kept(const or_spec* sp, long long q, long long key)
+{
+    long long s = sp->s;
+    switch (sp->family) {
+    case OR_DENSE:
+        return 1;
+    case OR_RADIAL:
+        return or_radial_kept(q / s, key / s, q % s, key % s, s);
+    case OR_WINDOW3D:
+        return or_window3d_kept(sp, q, key);
+    case OR_SWC:
+        return or_swc_kept(sp, q, key);
+    }
+    return 0;
+}
+
+/* Whole token mask (n x n bytes, row = query).  Small n only. */
+void oracle_dense_mask(const or_spec* sp, unsigned char* out)
+{
+    long long n = (long long)sp->f * sp->s;
+    for (long long q = 0; q < n; q++)
+        for (long long key = 0; key < n; key++)
+            out[q * n + key] = (unsigned char)oracle_kept(sp, q, key);
+}
+
+/* Number of kept pairs in the whole mask, by enumeration. */
+long long oracle_kept_total(const or_spec* sp)
+{
+    long long n = (long long)sp->f * sp->s, total = 0;
+#pragma omp parallel for reduction(+ : total) schedule(dynamic, 16)
+    for (long long q = 0; q < n; q++)
+        for (long long key = 0; key < n; key++)
+            total += oracle_kept(sp, q, key);
+    return total;
+}
+
+/* Kept-pair count of every tile (qb, kb) for the listed query tiles, by
+ * enumeration of every pair: out[r * nb + kb] for qbs[r]. */
+void oracle_tile_counts(const or_spec* sp, const int* qbs, int nq, int* out)
+{
+    long long n = (long long)sp->f * sp->s;
+    long long nb = (n + OR_TILE - 1) / OR_TILE;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < nq; r++) {
+        int* row = out + (long long)r * nb;
+        for (long long kb = 0; kb < nb; kb++)
+            row[kb] = 0;
+        for (long long q = (long long)qbs[r] * OR_TILE; q < (long long)(qbs[r] + 1) * OR_TILE && q < n; q++)
+            for (long long key = 0; key < n; key++)
+                if (oracle_kept(sp, q, key))
+                    row[key / OR_TILE] += 1;
+    }
+}
+
+/* Block-CSR from a full nb x nb count matrix: kept tiles of each row in
+ * ascending column order.  Returns nnz.  Pass null arrays to only count. */
+long long oracle_csr(const int* counts, long long n, int* row_ptr, int* col_idx, int* count,
+                     unsigned char* flag)
+{
+    long long nb = (n + OR_TILE - 1) / OR_TILE, nnz = 0;
+    for (long long qb = 0; qb < nb; qb++) {
+        if (row_ptr)
+            row_ptr[qb] = (int)nnz;
+        for (long long kb = 0; kb < nb; kb++) {
+            int c = counts[qb * nb + kb];
+            if (c > 0) {
+                if (col_idx) {
+                    col_idx[nnz] = (int)kb;
+                    count[nnz] = c;
+                    flag[nnz] = (c == OR_TILE * OR_TILE) ? OR_TILE_FULL : OR_TILE_PARTIAL;
+                }
+                nnz++;
+            }
+        }
+    }
+    if (row_ptr)
+        row_ptr[nb] = (int)nnz;
+    return nnz;
+}
+
+static double or_load(const void* base, int dtype, long long idx)
+{
+    if (dtype == OR_IN_BF16) {
+        uint32_t bits = (uint32_t)((const uint16_t*)base)[idx] << 16; /* bf16 is the top half of f32 */
+        float v;
+        memcpy(&v, &bits, sizeof v);
+        return (double)v;
+    }
+    if (dtype == OR_IN_F32)
+        return (double)((const float*)base)[idx];
+    return ((const double*)base)[idx];
+}
+
+/*
+ * Attention for a list of query rows ([RA] eq. 2 with M in {0,-inf}):
+ *   keys  = { key : M[q,key] == 0 }                    (token-exact mode)
+ *         = { key < n : tile (q/128, key/128) kept }  (block mode: kept tiles in full)
+ *   x     = scale * <Q[q], K[key]>,  p = exp(x - max x) / sum exp(x - max x)
+ *   O[q]  = sum p * V[key],  lse = log sum exp(x)
+ * Q, K, V are [B, H, n, d] row-major; row r is (row_bh[r] = b*H + h, row_q[r]).
+ * In block mode tile_flags[t * nb + kb] != 0 says tile (row_tile[r], kb) is
+ * kept, where t = row_tile_slot[r] indexes the caller's list of query tiles.
+ */
+void oracle_attention_rows(const void* Q, const void* K, const void* V, int dtype, long long n, int d,
+                           const or_spec* sp, int mode, double scale, long long nrows,
+                           const long long* row_bh, const long long* row_q,
+                           const unsigned char* tile_flags, const int* row_tile_slot, double* O,
+                           double* lse, long long* nkeys)
+{
+    long long nb = (n + OR_TILE - 1) / OR_TILE;
+#pragma omp parallel
+    {
+        double* x = (double*)malloc(sizeof(double) * (size_t)n);
+        long long* idx = (long long*)malloc(sizeof(long long) * (size_t)n);
+        double* acc = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 4)
+        for (long long r = 0; r < nrows; r++) {
+            long long q = row_q[r];
+            long long qoff = (row_bh[r] * n + q) * d;
+            long long kvbase = row_bh[r] * n * d;
+            long long m = 0;
+            for (long long key = 0; key < n; key++) {
+                int use;
+                if (mode == OR_TOKEN_EXACT)
+                    use = oracle_kept(sp, q, key);
+                else
+                    use = tile_flags[(long long)row_tile_slot[r] * nb + key / OR_TILE] != 0;
+                if (!use)
+                    continue;
+                double dot = 0.0;
+                for (int c = 0; c < d; c++)
+                    dot += or_load(Q, dtype, qoff + c) * or_load(K, dtype, kvbase + key * d + c);
+                x[m] = scale * dot;
+                idx[m] = key;
+                m++;
+            }
+            nkeys[r] = m;
+            if (m == 0) {
+                for (int c = 0; c < d; c++)
+                    O[r * d + c] = 0.0;
+                lse[r] = -INFINITY;
+                continue;
+            }
+            double mx = x[0];
+            for (long long t = 1; t < m; t++)
+                if (x[t] > mx)
+                    mx = x[t];
+            double denom = 0.0;
+            for (int c = 0; c < d; c++)
+                acc[c] = 0.0;
+            for (long long t = 0; t < m; t++) {
+                double w = exp(x[t] - mx);
+                denom += w;
+                for (int c = 0; c < d; c++)
+                    acc[c] += w * or_load(V, dtype, kvbase + idx[t] * d + c);
+            }
+            for (int c = 0; c < d; c++)
+                O[r * d + c] = acc[c] / denom;
+            lse[r] = mx + log(denom);
+        }
+        free(x);
+        free(idx);
+        free(acc);
+    }
+}
