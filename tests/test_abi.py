@@ -1,0 +1,110 @@
+"""The C ABI: the library loads, exports every declared entry point, and rejects
+bad arguments with the documented status before touching the GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "radattn.h")
+
+
+@pytest.fixture(scope="module")
+def ra():
+    from static_sparse_attention_b200 import build
+    build.build()
+    import static_sparse_attention_b200 as ra
+    return ra
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_]+\s*\**\s*(ra_[a-z0-9_]+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("ra_build_mask", "ra_attention_fwd", "ra_mask_info", "ra_mask_free", "ra_get_device_status",
+                 "ra_attention_fwd_host", "ra_status_string"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(ra):
+    lib = ctypes.CDLL(ra.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_version(ra):
+    assert ra.ra_status_string(ra.RA_OK) == b"ok"
+    assert ra.ra_status_string(ra.RA_ERR_DEVICE_TIMEOUT) == b"device wait timed out"
+    assert ra.ra_version() >= 10000
+
+
+def _build(ra, fam, f, s, params=None):
+    out = ctypes.c_void_p()
+    p = params or ra.ra_mask_params(0, 0, 0, 0, 0)
+    st = ra.ra_build_mask(fam, f, s, ctypes.byref(p), None, ctypes.byref(out))
+    return st, out
+
+
+@pytest.mark.parametrize("fam,f,s,params,status", [
+    (7, 4, 4, None, 1),                         # unknown family
+    (1, 0, 4, None, 1),                         # f < 1
+    (1, 4, 0, None, 1),                         # s < 1
+    (2, 4, 12, (3, 5, 1, 1, 0), 1),             # grid_h * grid_w != s
+    (2, 4, 12, (3, 4, -1, 1, 0), 1),            # negative radius
+    (3, 4, 12, (0, 0, 0, 0, 0), 1),             # window_frames < 1
+    (1, 1 << 20, 1 << 12, None, 2),             # n beyond the builder's limit
+])
+def test_build_mask_rejects_bad_arguments(ra, fam, f, s, params, status):
+    p = ra.ra_mask_params(*params) if params else None
+    st, out = _build(ra, fam, f, s, p)
+    assert st == status
+    assert not out.value
+    assert ra.ra_last_error()
+
+
+def test_build_mask_null_out(ra):
+    p = ra.ra_mask_params(0, 0, 0, 0, 0)
+    assert ra.ra_build_mask(1, 2, 2, ctypes.byref(p), None, None) == ra.RA_ERR_INVALID_ARG
+
+
+def test_attention_rejects_bad_arguments(ra):
+    fake = ctypes.c_void_p(0x10000)  # never dereferenced: validation fails first
+    args = dict(Q=0x10000, K=0x20000, V=0x30000, O=0x40000, B=1, H=1, d=128, m=fake, scale=0.1, mode=1)
+
+    def call(**kw):
+        a = {**args, **kw}
+        return ra.ra_attention_fwd(a["Q"], a["K"], a["V"], a["O"], a["B"], a["H"], a["d"], a["m"], a["scale"],
+                                   a["mode"], None, None)
+
+    assert call(Q=None) == ra.RA_ERR_INVALID_ARG
+    assert call(K=0x20008) == ra.RA_ERR_INVALID_ARG          # not 16-byte aligned
+    assert call(m=None) == ra.RA_ERR_INVALID_ARG
+    assert call(B=0) == ra.RA_ERR_INVALID_ARG
+    assert call(H=70000) == ra.RA_ERR_INVALID_ARG
+    assert call(d=96) == ra.RA_ERR_UNSUPPORTED
+    assert call(mode=5) == ra.RA_ERR_INVALID_ARG
+    assert call(scale=0.0) == ra.RA_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == ra.RA_ERR_INVALID_ARG
+    assert ra.ra_attention_fwd_host(None, None, None, None, None, None, None, None, 1, 1, 64, fake, 0.1, 1,
+                                    None) == ra.RA_ERR_INVALID_ARG
+
+
+def test_timeout_settings_are_range_checked(ra):
+    assert ra.ra_set_wait_timeout_ns(10) == ra.RA_ERR_INVALID_ARG
+    assert ra.ra_set_wait_timeout_ns(4_000_000_000) == ra.RA_OK
+    assert ra.ra_selftest_wait_timeout(5, None) == ra.RA_ERR_INVALID_ARG
+
+
+def test_product_path_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "static_sparse_attention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert "import oracle" not in text and "from oracle" not in text, fn
+                assert "radattn_oracle" not in text, fn

@@ -1,0 +1,172 @@
+"""GPU forward kernel vs the fp64 oracle on the same bf16 inputs.
+
+Bar: max |O_gpu - O_oracle| <= 1e-2 and ||O_gpu - O_oracle||_2 / ||O_oracle||_2
+<= 5e-3, on every row for the small configurations and on 256 seeded rows per
+head (boundary rows included) at full size, in the launch configuration the
+benchmark times."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import _gpu
+
+pytestmark = pytest.mark.gpu
+
+MODES = {"token_exact": oracle.TOKEN_EXACT, "block": oracle.BLOCK}
+
+
+def _run(spec: oracle.MaskSpec, Qh, Kh, Vh, mode: str, lse=False):
+    ra = _gpu.ra()
+    fam = {oracle.DENSE: "dense", oracle.RADIAL: "radial", oracle.WINDOW3D: "window3d", oracle.SWC: "swc"}[spec.family]
+    m = ra.Mask(fam, spec.f, spec.s, spec.grid_h, spec.grid_w, spec.r_t, spec.r_s, spec.window_frames)
+    q, k, v = (_gpu.to_device(t) for t in (Qh, Kh, Vh))
+    B, H, n, d = q.shape
+    out_lse = torch.empty((B, H, n), dtype=torch.float32, device="cuda") if lse else None
+    o = ra.attention_fwd(q, k, v, m, scale=_gpu.scale_for(d), mode=mode, lse=out_lse)
+    assert ra.device_status() == ra.RA_OK
+    return o, out_lse, m
+
+
+def _check(orc, spec, Qh, Kh, Vh, mode, rows=None, what=""):
+    o, lse, _ = _run(spec, Qh, Kh, Vh, mode, lse=True)
+    B, H, n, d = Qh.shape
+    row_bh, row_q = rows if rows is not None else _gpu.all_rows(B, H, n)
+    want, want_lse, nkeys = orc.attention_rows(Qh, Kh, Vh, spec, MODES[mode], _gpu.scale_for(d), row_bh, row_q)
+    got = _gpu.gather_rows(_gpu.to_f64(o), row_bh, row_q)
+    err = _gpu.assert_close(got, want, what)
+    got_lse = lse.cpu().numpy().astype(np.float64).reshape(B * H, n)[row_bh, row_q]
+    np.testing.assert_allclose(got_lse, want_lse, rtol=0, atol=2e-3, err_msg=f"{what}: lse")
+    return err
+
+
+# ------------------------------------------------------------ small configs
+
+def test_tiny_radial_token_exact_and_dense(orc):
+    _gpu.need_gpu()
+    c = synth.CONFIGS["tiny_radial"]
+    Q, K, V = synth.qkv_bf16("tiny_radial")
+    for mk in c["masks"]:
+        spec = oracle.spec_from(mk, c["f"], c["s"])
+        for mode in ("token_exact", "block"):
+            _check(orc, spec, Q, K, V, mode, what=f"tiny {mk['family']} {mode}")
+
+
+def test_tiny_fp32_originals_close_to_bf16_oracle(orc):
+    """The tiny config is generated in fp32; the GPU sees its bf16 rounding.  The
+    oracle on the fp32 originals stays within the bar of the GPU output too."""
+    _gpu.need_gpu()
+    c = synth.CONFIGS["tiny_radial"]
+    seed = synth.config_seed("tiny_radial")
+    shape = (c["B"], c["H"], c["f"] * c["s"], c["d"])
+    Qf, Kf, Vf = (synth.normal_f32(seed, t, shape) for t in range(3))
+    Qb, Kb, Vb = (synth.round_bf16(t) for t in (Qf, Kf, Vf))
+    spec = oracle.spec_from(c["masks"][0], c["f"], c["s"])
+    o, _, _ = _run(spec, Qb, Kb, Vb, "token_exact")
+    rows = _gpu.all_rows(1, 1, spec.n)
+    want32, _, _ = orc.attention_rows(Qf, Kf, Vf, spec, oracle.TOKEN_EXACT, _gpu.scale_for(c["d"]), *rows)
+    _gpu.assert_close(_gpu.gather_rows(_gpu.to_f64(o), *rows), want32, "tiny vs fp32 originals")
+
+
+@pytest.mark.parametrize("mk", synth.CONFIGS["window3d_16"]["masks"], ids=lambda m: f"rt{m['r_t']}_rs{m['r_s']}")
+@pytest.mark.parametrize("mode", ["token_exact", "block"])
+def test_window3d_all_rows(orc, mk, mode):
+    _gpu.need_gpu()
+    c = synth.CONFIGS["window3d_16"]
+    Q, K, V = synth.qkv_bf16("window3d_16")
+    spec = oracle.spec_from(mk, c["f"], c["s"], c["grid"])
+    _check(orc, spec, Q, K, V, mode, what=f"window3d {mk} {mode}")
+
+
+EDGE_CASES = [
+    # (family spec, B, H, d): ragged tails, n < 128, one frame, one token per frame
+    (oracle.MaskSpec(oracle.RADIAL, 11, 100), 1, 2, 128),
+    (oracle.MaskSpec(oracle.RADIAL, 1, 100), 2, 1, 64),
+    (oracle.MaskSpec(oracle.RADIAL, 1, 700), 1, 1, 128),
+    (oracle.MaskSpec(oracle.RADIAL, 300, 1), 1, 1, 64),
+    (oracle.MaskSpec(oracle.RADIAL, 37, 41), 3, 2, 64),
+    (oracle.MaskSpec(oracle.SWC, 9, 130, window_frames=3), 1, 3, 128),
+    (oracle.MaskSpec(oracle.WINDOW3D, 5, 99, 9, 11, 2, 4), 2, 1, 128),
+    (oracle.MaskSpec(oracle.DENSE, 3, 77), 1, 1, 64),
+    (oracle.MaskSpec(oracle.RADIAL, 64, 16), 1, 1, 128),   # sub-sampled diagonals (w > s)
+]
+
+
+@pytest.mark.parametrize("case", EDGE_CASES, ids=lambda c: f"fam{c[0].family}_f{c[0].f}_s{c[0].s}_B{c[1]}H{c[2]}d{c[3]}")
+@pytest.mark.parametrize("mode", ["token_exact", "block"])
+def test_edge_cases_all_rows(orc, case, mode):
+    _gpu.need_gpu()
+    spec, B, H, d = case
+    shape = (B, H, spec.n, d)
+    Q, K, V = (synth.normal_bf16(777, t, shape) for t in range(3))
+    _check(orc, spec, Q, K, V, mode, what=f"edge {case} {mode}")
+
+
+def test_invariants_on_gpu(orc):
+    """V = 1 gives O = 1; Q = 0 gives the mean of V over the kept keys."""
+    _gpu.need_gpu()
+    spec = oracle.MaskSpec(oracle.RADIAL, 11, 100)
+    shape = (1, 2, spec.n, 128)
+    Q, K, V = (synth.normal_bf16(99, t, shape) for t in range(3))
+    one = np.full(shape, 0x3F80, dtype=np.uint16)  # bf16 1.0
+    o, _, _ = _run(spec, Q, K, one, "token_exact")
+    assert np.abs(_gpu.to_f64(o) - 1.0).max() <= 1e-2
+    zero = np.zeros(shape, dtype=np.uint16)
+    o, _, _ = _run(spec, zero, K, V, "token_exact")
+    rows = _gpu.all_rows(1, 2, spec.n)
+    want, _, _ = orc.attention_rows(zero, K, V, spec, oracle.TOKEN_EXACT, 0.1, *rows)
+    _gpu.assert_close(_gpu.gather_rows(_gpu.to_f64(o), *rows), want, "Q = 0")
+
+
+def test_deterministic_bits():
+    _gpu.need_gpu()
+    spec = oracle.MaskSpec(oracle.RADIAL, 11, 100)
+    Q, K, V = (synth.normal_bf16(5, t, (1, 2, spec.n, 128)) for t in range(3))
+    a, _, _ = _run(spec, Q, K, V, "token_exact")
+    b, _, _ = _run(spec, Q, K, V, "token_exact")
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_host_io_entry_point_matches_device_call():
+    _gpu.need_gpu()
+    ra = _gpu.ra()
+    spec = oracle.MaskSpec(oracle.RADIAL, 11, 100)
+    shape = (1, 2, spec.n, 64)
+    Q, K, V = (synth.normal_bf16(6, t, shape) for t in range(3))
+    want, _, m = _run(spec, Q, K, V, "block")
+    hq, hk, hv = (torch.from_numpy(t.view(np.int16)).view(torch.bfloat16).pin_memory() for t in (Q, K, V))
+    ho = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+    dq, dk, dv, do = (torch.empty(shape, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    ra.attention_fwd_host(hq, hk, hv, ho, dq, dk, dv, do, m, mode="block")
+    torch.cuda.synchronize()
+    assert torch.equal(ho.view(torch.int16), want.cpu().view(torch.int16))
+
+
+def test_bounded_wait_selftest_reports_timeout():
+    """A kernel waits on an mbarrier nothing completes; its 20 ms bound expires and
+    the host reads RA_ERR_DEVICE_TIMEOUT; the context stays usable."""
+    _gpu.need_gpu()
+    ra = _gpu.ra()
+    assert ra.ra_selftest_wait_timeout(20_000_000, None) == ra.RA_ERR_DEVICE_TIMEOUT
+    assert ra.device_status() == ra.RA_OK
+    x = torch.ones(4, device="cuda")
+    assert float(x.sum()) == 4.0
+
+
+# ------------------------------------------------- full-size configs (sampled)
+
+FULL = [("wan_radial", 0, "block"), ("wan_radial", 1, "block"), ("hunyuan108k", 0, "block"),
+        ("hunyuan108k", 1, "block"), ("long460k", 0, "block"), ("hunyuan108k", 0, "token_exact")]
+
+
+@pytest.mark.parametrize("name,mask_i,mode", FULL, ids=lambda x: str(x))
+def test_full_size_sampled_rows(orc, name, mask_i, mode):
+    _gpu.need_gpu()
+    c = synth.CONFIGS[name]
+    Q, K, V = synth.qkv_bf16(name)
+    spec = oracle.spec_from(c["masks"][mask_i], c["f"], c["s"], c["grid"])
+    rows = _gpu.sampled_rows(synth.config_seed(name) ^ (mask_i + 1), c["f"], c["s"], c["B"], c["H"], 256)
+    _check(orc, spec, Q, K, V, mode, rows=rows, what=f"{name} {c['masks'][mask_i]} {mode}")
