@@ -170,6 +170,17 @@ ra_status ra_selftest_wait_timeout(long long timeout_ns, ra_stream stream);
 /* Limit of every bounded wait in the library's kernels (default 4e9 ns). */
 ra_status ra_set_wait_timeout_ns(long long timeout_ns);
 
+/* Precision of P in the P V product (process-wide setting).
+ *   RA_PV_AUTO   (default) bf16 P, except for masks whose rows average fewer
+ *                than 4096 computed keys: there P is held as a hi + lo pair of
+ *                bf16 numbers and P V runs as two MMAs, because over few keys the
+ *                rounding of each weight to bf16 is not averaged out.
+ *   RA_PV_BF16   always bf16 P (one MMA).
+ *   RA_PV_SPLIT  always hi + lo P (two MMAs).
+ * INVALID_ARG for any other value. */
+typedef enum { RA_PV_AUTO = 0, RA_PV_BF16 = 1, RA_PV_SPLIT = 2 } ra_pv_precision;
+ra_status ra_set_pv_precision(int policy);
+
 const char* ra_status_string(ra_status s);
 
 /* One-line description of the calling thread's last error ("" if none). */

@@ -8,7 +8,7 @@ that passes tensor addresses and the current CUDA stream.
 
 There is no CPU fallback: importing this package fails loudly when the
 compiled library is missing (build it with
-`python -m static_sparse_attention_b200.build`).
+`python static_sparse_attention_b200/build.py`).
 """
 from __future__ import annotations
 
@@ -20,7 +20,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libradattn.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libradattn.so is not built ({LIB_PATH}); run `python -m static_sparse_attention_b200.build`")
+    raise ImportError(f"libradattn.so is not built ({LIB_PATH}); run `python static_sparse_attention_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -30,6 +30,7 @@ RA_MODE_TOKEN_EXACT, RA_MODE_BLOCK = 0, 1
 RA_TILE_PARTIAL, RA_TILE_FULL = 0, 1
 RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_OUT_OF_MEMORY, RA_ERR_DEVICE_TIMEOUT = range(6)
 RA_TILE = 128
+RA_PV_AUTO, RA_PV_BF16, RA_PV_SPLIT = 0, 1, 2
 FAMILIES = {"dense": RA_MASK_DENSE, "radial": RA_MASK_RADIAL, "window3d": RA_MASK_WINDOW3D, "swc": RA_MASK_SWC}
 MODES = {"token_exact": RA_MODE_TOKEN_EXACT, "block": RA_MODE_BLOCK}
 
@@ -61,6 +62,7 @@ _SIGS = {
     "ra_get_device_error_site": ([ctypes.POINTER(_i), ctypes.POINTER(_i)], _i),
     "ra_selftest_wait_timeout": ([_ll, _vp], _i),
     "ra_set_wait_timeout_ns": ([_ll], _i),
+    "ra_set_pv_precision": ([_i], _i),
     "ra_status_string": ([_i], ctypes.c_char_p),
     "ra_last_error": ([], ctypes.c_char_p),
     "ra_version": ([], _i),

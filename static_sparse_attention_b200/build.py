@@ -1,6 +1,6 @@
 """Build libradattn.so in-tree: nvcc for sm_100a, static CUDA runtime.
 
-    python -m static_sparse_attention_b200.build [--force] [--verbose]
+    python static_sparse_attention_b200/build.py [--force] [--verbose]
 
 `--verbose` adds -Xptxas -v (registers, spills, shared memory per kernel).
 """

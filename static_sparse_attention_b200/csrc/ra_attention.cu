@@ -31,6 +31,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "ra_internal.h"
@@ -124,7 +125,10 @@ __device__ bool drain_wait(uint32_t bar, uint32_t parity, unsigned long long tim
     return true;
 }
 
-template <int D>
+// SPLIT_P: P is kept as hi + lo bf16 pairs (P = hi + lo to ~16 bits) and
+// P V runs as two MMAs; used for masks whose rows hold few keys, where the
+// rounding of P to bf16 is not averaged out over many keys.
+template <int D, bool SPLIT_P>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p)
@@ -243,6 +247,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         mma_ts(tmem + O_COL, tmem + sb * TILE + kk * 8,
                                smem_desc_sw128(vbase + kk * 2048, L::CHUNK_BYTES, 1024), idesc_pv,
                                (i > 0 || kk > 0) ? 1u : 0u);
+                    if (SPLIT_P) {
+#pragma unroll
+                        for (int kk = 0; kk < TILE / 16; ++kk)
+                            mma_ts(tmem + O_COL, tmem + sb * TILE + 64 + kk * 8,
+                                   smem_desc_sw128(vbase + kk * 2048, L::CHUNK_BYTES, 1024), idesc_pv, 1u);
+                    }
                     mma_commit(bar(B_V_EMPTY + st));
                     mma_commit(bar(B_S_FREE + sb));
                     mma_commit(bar(B_PV_DONE));
@@ -336,15 +346,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             float sum = 0.f;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t pk[16];
+                uint32_t pk[16], pl[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const float p0 = fast_exp2(fmaf(__uint_as_float(r[c][e]), p.scale_log2, -m_use));
                     const float p1 = fast_exp2(fmaf(__uint_as_float(r[c][e + 1]), p.scale_log2, -m_use));
                     sum += p0 + p1;
                     pk[e >> 1] = pack_bf16(p0, p1);
+                    if (SPLIT_P) {
+                        const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&pk[e >> 1]);
+                        pl[e >> 1] = pack_bf16(p0 - __low2float(hi), p1 - __high2float(hi));
+                    }
                 }
                 tmem_st16(lane_base + sb * TILE + c * 16, pk);
+                if (SPLIT_P)
+                    tmem_st16(lane_base + sb * TILE + 64 + c * 16, pl);
             }
             l_run += sum;
             tmem_wait_st();
@@ -449,22 +465,26 @@ ra_status make_map(CUtensorMap* map, const void* base, int BH, int n, int d)
     return RA_OK;
 }
 
-template <int D>
+template <int D, bool SPLIT_P>
 ra_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p, int B,
                      cudaStream_t cs)
 {
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(attn_fwd_kernel<D, SPLIT_P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         Layout<D>::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess)
         return cuda_fail(attr_err, "cudaFuncSetAttribute(attn_fwd_kernel)");
     dim3 grid(p.nb, p.H, B);
-    attn_fwd_kernel<D><<<grid, NUM_THREADS, Layout<D>::SMEM_BYTES, cs>>>(mq, mk, mv, p);
+    attn_fwd_kernel<D, SPLIT_P><<<grid, NUM_THREADS, Layout<D>::SMEM_BYTES, cs>>>(mq, mk, mv, p);
     return cuda_fail(cudaGetLastError(), "attn_fwd_kernel launch");
 }
+
+// Rows averaging fewer computed keys than this use the split-P kernel.
+constexpr long long SPLIT_P_MAX_KEYS_PER_ROW = 4096;
+std::atomic<int> g_pv_policy{RA_PV_AUTO};
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
@@ -529,7 +549,13 @@ extern "C" ra_status ra_attention_fwd(const void* Q, const void* K, const void* 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = wait_timeout_ns();
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    return d == 64 ? launch_fwd<64>(mq, mk, mv, p, B, cs) : launch_fwd<128>(mq, mk, mv, p, B, cs);
+    const long long pairs = mode == RA_MODE_BLOCK ? m->block_pairs : m->kept_pairs;
+    const int policy = g_pv_policy.load(std::memory_order_relaxed);
+    const bool split = policy == RA_PV_SPLIT ||
+                       (policy == RA_PV_AUTO && pairs < SPLIT_P_MAX_KEYS_PER_ROW * static_cast<long long>(n));
+    if (d == 64)
+        return split ? launch_fwd<64, true>(mq, mk, mv, p, B, cs) : launch_fwd<64, false>(mq, mk, mv, p, B, cs);
+    return split ? launch_fwd<128, true>(mq, mk, mv, p, B, cs) : launch_fwd<128, false>(mq, mk, mv, p, B, cs);
 }
 
 extern "C" ra_status ra_attention_fwd_host(const void* Q_host, const void* K_host, const void* V_host, void* O_host,
@@ -586,4 +612,12 @@ extern "C" ra_status ra_selftest_wait_timeout(long long timeout_ns, ra_stream st
     wait_selftest_kernel<<<1, 32, 0, cs>>>(static_cast<unsigned long long>(timeout_ns));
     RA_CUDA_TRY(cudaGetLastError());
     return ra_get_device_status(stream);
+}
+
+extern "C" ra_status ra_set_pv_precision(int policy)
+{
+    if (policy != RA_PV_AUTO && policy != RA_PV_BF16 && policy != RA_PV_SPLIT)
+        return fail(RA_ERR_INVALID_ARG, "unknown P precision policy %d", policy);
+    g_pv_policy.store(policy, std::memory_order_relaxed);
+    return RA_OK;
 }

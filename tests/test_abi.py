@@ -12,8 +12,8 @@ HEADER = os.path.join(ROOT, "include", "radattn.h")
 
 @pytest.fixture(scope="module")
 def ra():
-    from static_sparse_attention_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import static_sparse_attention_b200 as ra
     return ra
 
@@ -98,6 +98,8 @@ def test_timeout_settings_are_range_checked(ra):
     assert ra.ra_set_wait_timeout_ns(10) == ra.RA_ERR_INVALID_ARG
     assert ra.ra_set_wait_timeout_ns(4_000_000_000) == ra.RA_OK
     assert ra.ra_selftest_wait_timeout(5, None) == ra.RA_ERR_INVALID_ARG
+    assert ra.ra_set_pv_precision(7) == ra.RA_ERR_INVALID_ARG
+    assert ra.ra_set_pv_precision(ra.RA_PV_AUTO) == ra.RA_OK
 
 
 def test_product_path_does_not_import_the_oracle():

@@ -95,14 +95,24 @@ EDGE_CASES = [
 ]
 
 
+@pytest.fixture
+def pv_policy(request):
+    ra = _gpu.ra()
+    ra.check(ra.ra_set_pv_precision(request.param), "ra_set_pv_precision")
+    yield request.param
+    ra.ra_set_pv_precision(ra.RA_PV_AUTO)
+
+
 @pytest.mark.parametrize("case", EDGE_CASES, ids=lambda c: f"fam{c[0].family}_f{c[0].f}_s{c[0].s}_B{c[1]}H{c[2]}d{c[3]}")
 @pytest.mark.parametrize("mode", ["token_exact", "block"])
-def test_edge_cases_all_rows(orc, case, mode):
+@pytest.mark.parametrize("pv_policy", [1, 2], ids=["bf16P", "splitP"], indirect=True)
+def test_edge_cases_all_rows(orc, case, mode, pv_policy):
+    """Both P paths (one bf16 MMA, hi + lo MMAs) on every edge case."""
     _gpu.need_gpu()
     spec, B, H, d = case
     shape = (B, H, spec.n, d)
     Q, K, V = (synth.normal_bf16(777, t, shape) for t in range(3))
-    _check(orc, spec, Q, K, V, mode, what=f"edge {case} {mode}")
+    _check(orc, spec, Q, K, V, mode, what=f"edge {case} {mode} pv={pv_policy}")
 
 
 def test_invariants_on_gpu(orc):
