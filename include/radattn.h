@@ -111,6 +111,35 @@ typedef struct {
 ra_status ra_build_mask(int family, int f, int s, const ra_mask_params* params, ra_stream stream,
                         ra_mask** out);
 
+/*
+ * ra_build_mask_noalloc -- ra_build_mask for callers that cannot allocate.
+ * (No counterpart in the paper: this is a deployment variant of the builder.)
+ *
+ * Some callers must not have a library allocate device memory behind their
+ * back: engines whose own allocator owns the whole device, processes that
+ * reserve a fixed memory budget at start-up, and loops that cannot afford the
+ * device-wide synchronisation an allocation may imply.  This entry point builds
+ * the same block-CSR as ra_build_mask into arrays the caller supplies and calls
+ * no allocating routine.  Its scratch (the tile counts and row statistics) is a
+ * fixed array of 4 MiB + 4.25 KiB compiled into the library, which every device
+ * that loads the library holds until the process exits.
+ *   row_ptr               : device int32[nb + 1], written.
+ *   col_idx, count, flag  : device int32 / int32 / uint8 arrays of nnz_capacity
+ *                           entries, written with the kept tiles.
+ *   info                  : optional host struct, filled even when the capacity
+ *                           is too small (so the caller can size the arrays).
+ * Limit: n <= 131072 tokens (nb <= 1024); larger masks get RA_ERR_UNSUPPORTED.
+ * RA_ERR_INVALID_ARG if nnz exceeds nnz_capacity (nothing but row_ptr written).
+ * Synchronises `stream` once (to read nnz).  The first call on a device looks up
+ * the scratch's device address and may load the library's module on that
+ * device: make it before any stream capture.  All calls share the one scratch
+ * array, so calls that can overlap on the GPU (different streams, no ordering)
+ * race; calls ordered on one stream are safe.
+ */
+ra_status ra_build_mask_noalloc(int family, int f, int s, const ra_mask_params* params, int* row_ptr, int* col_idx,
+                                int* count, unsigned char* flag, long long nnz_capacity, ra_mask_info_t* info,
+                                ra_stream stream);
+
 /* Fill *info.  Host only, no synchronisation. */
 ra_status ra_mask_info(const ra_mask* m, ra_mask_info_t* info);
 

@@ -52,6 +52,8 @@ _MaskP = ctypes.c_void_p
 _SIGS = {
     "ra_build_mask": ([_i, _i, _i, ctypes.POINTER(ra_mask_params), _vp, ctypes.POINTER(_MaskP)], _i),
     "ra_mask_info": ([_MaskP, ctypes.POINTER(ra_mask_info_t)], _i),
+    "ra_build_mask_noalloc": ([_i, _i, _i, ctypes.POINTER(ra_mask_params), _vp, _vp, _vp, _vp, _ll,
+                               ctypes.POINTER(ra_mask_info_t), _vp], _i),
     "ra_mask_copy_to_host": ([_MaskP, _vp, _vp, _vp, _vp], _i),
     "ra_mask_device_arrays": ([_MaskP, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
                                ctypes.POINTER(_vp)], _i),

@@ -19,6 +19,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "ra_internal.h"
 
@@ -175,6 +176,26 @@ __global__ void __launch_bounds__(128) compact_kernel(const int* __restrict__ co
         out += chunk;
         __syncthreads();
     }
+}
+
+// ---------------------------------------------------------------------------
+// Scratch of ra_build_mask_noalloc.  Some callers cannot allocate device memory
+// on demand (see the header); for them the builder's scratch -- the nb x nb
+// tile counts, the per-row kept-tile counts and the statistics -- lives in this
+// file-scope array, reserved on every device that loads the library.
+constexpr int NOALLOC_MAX_NB = 1024;  // n <= 131072 tokens
+constexpr size_t NOALLOC_COUNTS_BYTES = sizeof(int) * static_cast<size_t>(NOALLOC_MAX_NB) * NOALLOC_MAX_NB;
+constexpr size_t NOALLOC_ROWS_BYTES = sizeof(int) * NOALLOC_MAX_NB;
+constexpr size_t NOALLOC_SCRATCH_BYTES = NOALLOC_COUNTS_BYTES + NOALLOC_ROWS_BYTES + 256;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+__global__ void init_totals_kernel(BuildTotals* tot)
+{
+    tot->kept_pairs = 0;
+    tot->block_pairs = 0;
+    tot->full_tiles = 0;
+    tot->row_min = INT_MAX;
+    tot->row_max = 0;
 }
 
 void free_mask_arrays(ra_mask* m)
@@ -376,4 +397,84 @@ extern "C" void ra_mask_free(ra_mask* m)
     cudaDeviceSynchronize();
     free_mask_arrays(m);
     delete m;
+}
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device (host code cannot use the symbol itself as a device address).
+static ra_status noalloc_scratch_address(unsigned char** out)
+{
+    static std::mutex mu;
+    static unsigned char* addr[128] = {};
+    int dev = 0;
+    RA_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 128)
+        return fail(RA_ERR_UNSUPPORTED, "device ordinal %d is beyond the library's table", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaGetSymbolAddress(builder scratch)");
+        addr[dev] = static_cast<unsigned char*>(p);
+    }
+    *out = addr[dev];
+    return RA_OK;
+}
+
+extern "C" ra_status ra_build_mask_noalloc(int family, int f, int s, const ra_mask_params* params, int* row_ptr,
+                                           int* col_idx, int* count, unsigned char* flag, long long nnz_capacity,
+                                           ra_mask_info_t* info, ra_stream stream)
+{
+    MaskGeom g;
+    ra_status st = validate_geometry(family, f, s, params, &g);
+    if (st != RA_OK)
+        return st;
+    const int nb = (g.n + TILE - 1) / TILE;
+    if (nb > NOALLOC_MAX_NB)
+        return fail(RA_ERR_UNSUPPORTED,
+                    "ra_build_mask_noalloc handles at most %d x 128 = %d tokens (its fixed scratch); n = %d",
+                    NOALLOC_MAX_NB, NOALLOC_MAX_NB * TILE, g.n);
+    if (!row_ptr || (nnz_capacity > 0 && (!col_idx || !count || !flag)) || nnz_capacity < 0)
+        return fail(RA_ERR_INVALID_ARG, "NULL output array or negative capacity");
+    unsigned char* scratch = nullptr;
+    if ((st = noalloc_scratch_address(&scratch)) != RA_OK)
+        return st;
+    int* counts = reinterpret_cast<int*>(scratch);
+    int* row_tiles = reinterpret_cast<int*>(scratch + NOALLOC_COUNTS_BYTES);
+    BuildTotals* tot = reinterpret_cast<BuildTotals*>(scratch + NOALLOC_COUNTS_BYTES + NOALLOC_ROWS_BYTES);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+    // The scratch keeps the previous call's contents: the statistics start from
+    // zero here; every count and per-row entry used below is rewritten.
+    init_totals_kernel<<<1, 1, 0, cs>>>(tot);
+    RA_CUDA_TRY(cudaGetLastError());
+    tile_count_kernel<<<nb, TILE, 0, cs>>>(g, nb, counts, row_tiles, tot);
+    RA_CUDA_TRY(cudaGetLastError());
+    row_scan_kernel<<<1, 1024, 0, cs>>>(row_tiles, nb, row_ptr);
+    RA_CUDA_TRY(cudaGetLastError());
+    BuildTotals h;
+    int nnz = 0;
+    RA_CUDA_TRY(cudaMemcpyAsync(&h, tot, sizeof h, cudaMemcpyDeviceToHost, cs));
+    RA_CUDA_TRY(cudaMemcpyAsync(&nnz, row_ptr + nb, sizeof nnz, cudaMemcpyDeviceToHost, cs));
+    RA_CUDA_TRY(cudaStreamSynchronize(cs));
+    if (info) {
+        info->family = g.family;
+        info->f = g.f;
+        info->s = g.s;
+        info->nb = nb;
+        info->n = g.n;
+        info->nnz = nnz;
+        info->full_tiles = static_cast<long long>(h.full_tiles);
+        info->kept_pairs = static_cast<long long>(h.kept_pairs);
+        info->block_pairs = static_cast<long long>(h.block_pairs);
+        info->row_min = h.row_min;
+        info->row_max = h.row_max;
+    }
+    if (nnz > nnz_capacity)
+        return fail(RA_ERR_INVALID_ARG, "the mask keeps %d tiles but the output arrays hold %lld", nnz, nnz_capacity);
+    if (nnz > 0) {
+        compact_kernel<<<nb, TILE, 0, cs>>>(counts, nb, row_ptr, col_idx, count, flag);
+        RA_CUDA_TRY(cudaGetLastError());
+    }
+    return RA_OK;
 }
