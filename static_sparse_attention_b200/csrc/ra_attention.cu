@@ -7,31 +7,41 @@
 // applies the element mask; in block mode every valid pair of a kept tile is
 // used.  Keys >= n are masked in both modes; rows >= n are never stored.
 //
-// One CTA per query tile, 6 warps with fixed roles:
-//   warps 0-3  softmax: thread t owns query row t (TMEM lane t); reads S from
-//              TMEM, masks, keeps a running max / sum, writes P (bf16) back to
-//              TMEM over S, rescales O in TMEM when the max grows by > 2^8,
-//              and runs the epilogue O / l -> bf16.
-//   warp 4     producer: one thread issues TMA loads of Q once and of the K / V
-//              tiles of the row into two-stage rings (128-byte swizzle).
-//   warp 5     MMA: allocates 512 TMEM columns; one thread issues
-//              S_j = Q K_j^T (tcgen05.mma, A and B from shared memory) into one of
-//              three S buffers, and O += P_j V_j (A = P from TMEM, B = V from
-//              shared memory); completion is signalled by tcgen05.commit.
-// TMEM columns: S buffers at 0, 128, 256 (fp32, 128 columns each; P overlays
-// the first 64 columns as packed bf16 pairs), O at 384 (fp32, d columns).
+// One CTA per query tile, two CTAs resident per SM (256 TMEM columns, under
+// half the shared memory each).  Keys move in half-tiles of 64: half-tile h of
+// the row is half h % 2 of kept tile h / 2.  192 threads in fixed roles:
+//   warps 0-3  softmax: thread t owns query row t (TMEM lane t); per half-tile
+//              reads S from TMEM, masks, keeps the running max / sum, writes P
+//              (bf16) back over S, and at the end runs the epilogue O / l.
+//   warp 4     producer: TMA loads of Q once, then the K and V half-tiles of
+//              the row into two rings (128-byte swizzle).
+//   warp 5     MMA: allocates TMEM; one thread issues S_h = Q K_h^T
+//              (tcgen05.mma, N = 64) into S buffer h % 2 and O += P_h V_h
+//              (A = P from TMEM), in the order S_0, S_1, PV_0, S_2, PV_1, ...:
+//              S of the next half-tile is in flight while the softmax works on
+//              the current one.
+// TMEM columns: S buffers at 0 and 64 (fp32, 64 columns; P overlays each as
+// packed bf16), O at 128 (fp32, d columns).
+//
+// tcgen05 MMAs issued by one thread execute in issue order, and a commit
+// arrives once every earlier MMA of the thread has completed; so S_{h+2} may
+// overwrite the P_h that PV_h reads (it is issued after it).  The softmax
+// rescales O only after the P V of the previous half-tile has completed.
 //
 // Online softmax in base 2: x = S * scale * log2(e); p = 2^(x - m) with m a
-// running maximum that is only raised (and O, l rescaled) when a tile's maximum
-// exceeds it by more than 8; p <= 2^8 otherwise, which fp32 and bf16 hold
-// exactly as well as p <= 1, and O / l is independent of the reference m.
+// running maximum that is only raised (and O, l rescaled) when a half-tile's
+// maximum exceeds it by more than 8; p <= 2^8 otherwise, which fp32 and bf16
+// hold with the same relative precision as p <= 1, and O / l does not depend on
+// m.  After the first half-tile the exponentials are computed against the
+// running maximum in the same pass that finds the half-tile's maximum.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+#include <climits>
 #include <cmath>
 #include <cstring>
-#include <atomic>
 #include <mutex>
 
 #include "ra_internal.h"
@@ -45,47 +55,51 @@ __device__ int g_err[4];
 namespace {
 
 constexpr int NUM_THREADS = 192;
-constexpr int KV_STAGES = 2;
-constexpr int S_BUFS = 3;
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t O_COL = 384;
+constexpr uint32_t TMEM_COLS = 256;
+// Keys per half-tile: K, V, S and P move 64 keys at a time.
+constexpr int HALF = 64;
+// TMEM columns of S / P buffer `buf` (64 fp32 columns) and of O (d fp32 columns).
+__host__ __device__ constexpr uint32_t s_col_of(int buf) { return 64u * static_cast<uint32_t>(buf); }
+constexpr uint32_t O_COL = 128;
 constexpr float RESCALE_THRESHOLD = 8.0f;
 
 // Wait-site codes recorded with a timeout.
 enum : int {
-    SITE_Q_FULL = 1, SITE_K_EMPTY, SITE_V_EMPTY, SITE_S_FREE, SITE_K_FULL, SITE_P_FULL, SITE_V_FULL,
-    SITE_S_FULL, SITE_PV_DONE, SITE_O_FINAL, SITE_DRAIN, SITE_SELFTEST
+    SITE_Q_FULL = 1, SITE_K_EMPTY, SITE_V_EMPTY, SITE_K_FULL, SITE_P_FULL, SITE_V_FULL, SITE_S_FULL,
+    SITE_PV_DONE, SITE_O_FINAL, SITE_SELFTEST, SITE_SMEM_ALIGN
 };
 
 template <int D>
 struct Layout {
-    static constexpr int CHUNKS = D / 64;                  // 128-byte swizzle atoms across d
-    static constexpr int CHUNK_BYTES = TILE * 128;          // 128 rows x 128 bytes
-    static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES; // one 128 x d bf16 tile
+    static constexpr int CHUNKS = D / 64;                          // 128-byte swizzle atoms across d
+    static constexpr int Q_CHUNK_BYTES = TILE * 128;                // 128 rows x 128 bytes
+    static constexpr int Q_BYTES = CHUNKS * Q_CHUNK_BYTES;          // the 128 x d query tile
+    static constexpr int H_CHUNK_BYTES = HALF * 128;                // 64 rows x 128 bytes
+    static constexpr int H_BYTES = CHUNKS * H_CHUNK_BYTES;          // a 64 x d half-tile of K or V
+    static constexpr int KS = D == 64 ? 4 : 3;                      // K ring stages (half-tiles)
+    static constexpr int VS = D == 64 ? 4 : 2;                      // V ring stages (half-tiles)
     static constexpr int Q_OFF = 0;
-    static constexpr int K_OFF = Q_OFF + TILE_BYTES;
-    static constexpr int V_OFF = K_OFF + KV_STAGES * TILE_BYTES;
-    static constexpr int BAR_OFF = V_OFF + KV_STAGES * TILE_BYTES;
+    static constexpr int K_OFF = Q_OFF + Q_BYTES;
+    static constexpr int V_OFF = K_OFF + KS * H_BYTES;
+    static constexpr int BAR_OFF = V_OFF + VS * H_BYTES;
     static constexpr int BAR_BYTES = 256;
-    // + alignment slack; at least 120 KB so that one CTA (and its 512 TMEM
-    // columns) owns the SM.
-    static constexpr int SMEM_NEEDED = BAR_OFF + BAR_BYTES + 1024;
-    static constexpr int SMEM_BYTES = SMEM_NEEDED > 120 * 1024 ? SMEM_NEEDED : 120 * 1024;
+    // Two CTAs share an SM; the dynamic shared memory is 1024-byte aligned
+    // (checked at run time) so no alignment slack is reserved.
+    static constexpr int SMEM_BYTES = BAR_OFF + BAR_BYTES;
 };
 
 // Barrier slots (8 bytes each) inside the barrier region.
 enum : int {
     B_Q_FULL = 0,
-    B_K_FULL = 1,       // + stage
-    B_K_EMPTY = 3,      // + stage
-    B_V_FULL = 5,       // + stage
-    B_V_EMPTY = 7,      // + stage
-    B_S_FULL = 9,       // + buffer
-    B_P_FULL = 12,      // + buffer
-    B_S_FREE = 15,      // + buffer
-    B_PV_DONE = 18,
-    B_O_FINAL = 19,
-    B_COUNT = 20
+    B_K_FULL = 1,    // + stage (up to 4)
+    B_K_EMPTY = 5,   // + stage
+    B_V_FULL = 9,    // + stage
+    B_V_EMPTY = 13,  // + stage
+    B_S_FULL = 17,   // + buffer
+    B_P_FULL = 19,   // + buffer
+    B_PV_DONE = 21,
+    B_O_FINAL = 22,
+    B_COUNT = 23
 };
 
 struct FwdParams {
@@ -113,6 +127,116 @@ __device__ __forceinline__ float fast_exp2(float x)
     return y;
 }
 
+// ---- packed fp32 pairs (sm_100 f32x2 instructions) -------------------------
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair of values on the FMA pipe instead of MUFU.  Range reduction
+// x = j + f with j = round(x) (by the 1.5 * 2^23 rounding constant) and
+// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial (Remez fit of the relative
+// error, coefficients from exp2_poly_fit.py, max relative error 7.5e-5); 2^j
+// added to the exponent field.  x is clamped at -126, so the result is
+// a tiny positive number (not 0) below 2^-126: only used on unmasked tiles.
+constexpr float EXP2_C0 = 0.99992806f, EXP2_C1 = 0.69326097f, EXP2_C2 = 0.24261113f, EXP2_C3 = 0.05517167f;
+__device__ __forceinline__ void poly_exp2_x2(float x0, float x1, float& y0, float& y1)
+{
+    const float rnd = 12582912.0f;  // 1.5 * 2^23
+    x0 = fmaxf(x0, -126.0f);
+    x1 = fmaxf(x1, -126.0f);
+    const uint64_t x = f2pack(x0, x1);
+    const uint64_t r = f2add(x, f2pack(rnd, rnd));               // j in the low mantissa bits
+    const uint64_t j = f2add(r, f2pack(-rnd, -rnd));
+    const uint64_t f = f2fma(j, f2pack(-1.0f, -1.0f), x);         // x - j
+    uint64_t poly = f2fma(f2pack(EXP2_C3, EXP2_C3), f, f2pack(EXP2_C2, EXP2_C2));
+    poly = f2fma(poly, f, f2pack(EXP2_C1, EXP2_C1));
+    poly = f2fma(poly, f, f2pack(EXP2_C0, EXP2_C0));
+    float p0, p1, r0, r1;
+    f2unpack(poly, p0, p1);
+    f2unpack(r, r0, r1);
+    // (bits of r) << 23 == j << 23 modulo 2^32, since 0x4B400000 << 23 wraps to 0.
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(r0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(r1) << 23));
+}
+
+// Exponentials, bf16 packing and row sums of one 32-column chunk of S:
+// p = 2^(s * c - m).  The first EMU elements of the chunk use the polynomial,
+// the rest MUFU ex2.  The row sum is kept in SUMACC independent accumulators
+// (short dependency chains).  SPLIT also returns the bf16 residuals.
+#ifndef RA_SUMACC
+#define RA_SUMACC 8
+#endif
+#ifndef RA_MAXACC
+#define RA_MAXACC 8
+#endif
+#ifndef RA_FFMA2
+#define RA_FFMA2 0
+#endif
+template <int EMU, bool SPLIT, bool MAX>
+__device__ __forceinline__ void exp_chunk(const uint32_t (&r)[32], float c, float negm, float (&acc)[RA_SUMACC],
+                                          float (&mx)[4], uint32_t (&pk)[16], uint32_t (&pl)[16])
+{
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        if (MAX)
+            mx[(e >> 1) & 3] = max3(mx[(e >> 1) & 3], __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+        float x0, x1, p0, p1;
+        if (RA_FFMA2) {
+            const uint64_t x2 = f2fma(f2pack(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), f2pack(c, c),
+                                      f2pack(negm, negm));
+            f2unpack(x2, x0, x1);
+        } else {
+            x0 = fmaf(__uint_as_float(r[e]), c, negm);
+            x1 = fmaf(__uint_as_float(r[e + 1]), c, negm);
+        }
+        if (e < EMU) {
+            poly_exp2_x2(x0, x1, p0, p1);
+        } else {
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
+        }
+        acc[(e >> 1) % RA_SUMACC] += p0 + p1;
+        pk[e >> 1] = pack_bf16(p0, p1);
+        if (SPLIT) {
+            const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&pk[e >> 1]);
+            pl[e >> 1] = pack_bf16(p0 - __low2float(hi), p1 - __high2float(hi));
+        }
+    }
+}
+
+// Elements of each 32-column chunk whose exponential runs on the FMA pipe
+// (unmasked tiles, bf16 P only): shifts work off the MUFU unit, which at
+// d = 128 needs as many cycles per tile as the tensor core.
+#ifndef RA_EMU_PER_32
+#define RA_EMU_PER_32 0
+#endif
+constexpr int EMU_PER_32 = RA_EMU_PER_32;
+
 // Wait without the CTA abort flag: used only to drain in-flight copies and
 // MMAs before the CTA releases its memory.
 __device__ bool drain_wait(uint32_t bar, uint32_t parity, unsigned long long timeout_ns)
@@ -129,16 +253,13 @@ __device__ bool drain_wait(uint32_t bar, uint32_t parity, unsigned long long tim
 // P V runs as two MMAs; used for masks whose rows hold few keys, where the
 // rounding of P to bf16 is not averaged out over many keys.
 template <int D, bool SPLIT_P>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(NUM_THREADS, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p)
 {
     using L = Layout<D>;
-    extern __shared__ uint8_t smem_raw[];
-    // 1024-byte alignment for the 128-byte-swizzled tiles.
-    const uint32_t raw_addr = smem_addr(smem_raw);
-    const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
-    uint8_t* smem = smem_raw + (sbase - raw_addr);
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sbase = smem_addr(smem);
     const uint32_t sQ = sbase + L::Q_OFF, sK = sbase + L::K_OFF, sV = sbase + L::V_OFF;
     const uint32_t bars = sbase + L::BAR_OFF;
     auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
@@ -153,8 +274,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (threadIdx.x == 0) {
         *abort_flag = *reinterpret_cast<volatile int*>(g_err) != 0 ? 1 : 0;
+        if (sbase & 1023u)  // the swizzled tiles need 1024-byte alignment: record it, run nothing
+            report_timeout(wc, SITE_SMEM_ALIGN);
         for (int i = 0; i < B_COUNT; ++i)
-            mbar_init(bar(i), (i >= B_P_FULL && i < B_P_FULL + S_BUFS) ? 128u : 1u);
+            mbar_init(bar(i), (i == B_P_FULL || i == B_P_FULL + 1) ? 128u : 1u);
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -170,6 +293,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     const int row_start = p.row_ptr[qb];
     const int L_row = skip ? 0 : p.row_ptr[qb + 1] - row_start;
+    const int n_half = 2 * L_row;
 
     if (warp == 4) {
         // ------------------------------------------------------------ producer
@@ -177,84 +301,83 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_prefetch_map(&tmQ);
             tma_prefetch_map(&tmK);
             tma_prefetch_map(&tmV);
-            mbar_arrive_expect_tx(bar(B_Q_FULL), L::TILE_BYTES);
+            mbar_arrive_expect_tx(bar(B_Q_FULL), L::Q_BYTES);
             for (int c = 0; c < L::CHUNKS; ++c)
-                tma_load_3d(sQ + c * L::CHUNK_BYTES, &tmQ, bar(B_Q_FULL), c * 64, qb * TILE, bh);
+                tma_load_3d(sQ + c * L::Q_CHUNK_BYTES, &tmQ, bar(B_Q_FULL), c * 64, qb * TILE, bh);
             int k_issued = 0, v_issued = 0;
-            for (int j = 0; j < L_row; ++j) {
-                const int st = j & 1;
-                const int kb = p.col_idx[row_start + j];
-                if (j >= KV_STAGES && !mbar_wait(bar(B_K_EMPTY + st), ((j >> 1) - 1) & 1, wc, SITE_K_EMPTY))
+            for (int hh = 0; hh < n_half; ++hh) {
+                const int key0 = p.col_idx[row_start + (hh >> 1)] * TILE + (hh & 1) * HALF;
+                const int ks = hh % L::KS, vs = hh % L::VS;
+                if (hh >= L::KS && !mbar_wait(bar(B_K_EMPTY + ks), ((hh / L::KS) - 1) & 1, wc, SITE_K_EMPTY))
                     break;
-                mbar_arrive_expect_tx(bar(B_K_FULL + st), L::TILE_BYTES);
+                mbar_arrive_expect_tx(bar(B_K_FULL + ks), L::H_BYTES);
                 for (int c = 0; c < L::CHUNKS; ++c)
-                    tma_load_3d(sK + st * L::TILE_BYTES + c * L::CHUNK_BYTES, &tmK, bar(B_K_FULL + st), c * 64,
-                                kb * TILE, bh);
-                k_issued = j + 1;
-                if (j >= KV_STAGES && !mbar_wait(bar(B_V_EMPTY + st), ((j >> 1) - 1) & 1, wc, SITE_V_EMPTY))
+                    tma_load_3d(sK + ks * L::H_BYTES + c * L::H_CHUNK_BYTES, &tmK, bar(B_K_FULL + ks), c * 64,
+                                key0, bh);
+                k_issued = hh + 1;
+                if (hh >= L::VS && !mbar_wait(bar(B_V_EMPTY + vs), ((hh / L::VS) - 1) & 1, wc, SITE_V_EMPTY))
                     break;
-                mbar_arrive_expect_tx(bar(B_V_FULL + st), L::TILE_BYTES);
+                mbar_arrive_expect_tx(bar(B_V_FULL + vs), L::H_BYTES);
                 for (int c = 0; c < L::CHUNKS; ++c)
-                    tma_load_3d(sV + st * L::TILE_BYTES + c * L::CHUNK_BYTES, &tmV, bar(B_V_FULL + st), c * 64,
-                                kb * TILE, bh);
-                v_issued = j + 1;
+                    tma_load_3d(sV + vs * L::H_BYTES + c * L::H_CHUNK_BYTES, &tmV, bar(B_V_FULL + vs), c * 64,
+                                key0, bh);
+                v_issued = hh + 1;
             }
             // Let every copy this thread issued land before the CTA can exit.  A
             // load into a stage is issued only after the previous load of that
             // stage was consumed, so only the last load of each stage can be in
             // flight here, and its phase parity identifies it.
             drain_wait(bar(B_Q_FULL), 0, p.timeout_ns);
-            for (int j = max(0, k_issued - KV_STAGES); j < k_issued; ++j)
-                drain_wait(bar(B_K_FULL + (j & 1)), (j >> 1) & 1, p.timeout_ns);
-            for (int j = max(0, v_issued - KV_STAGES); j < v_issued; ++j)
-                drain_wait(bar(B_V_FULL + (j & 1)), (j >> 1) & 1, p.timeout_ns);
+            for (int j = max(0, k_issued - L::KS); j < k_issued; ++j)
+                drain_wait(bar(B_K_FULL + j % L::KS), (j / L::KS) & 1, p.timeout_ns);
+            for (int j = max(0, v_issued - L::VS); j < v_issued; ++j)
+                drain_wait(bar(B_V_FULL + j % L::VS), (j / L::VS) & 1, p.timeout_ns);
         }
     } else if (warp == 5) {
         // ----------------------------------------------------------------- MMA
         if (lane == 0 && L_row > 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, TILE, 0, 0);
+            constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, HALF, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(TILE, D, 0, 1);
             bool ok = mbar_wait(bar(B_Q_FULL), 0, wc, SITE_Q_FULL);
             tc_fence_after();
-            for (int j = 0; ok && j <= L_row; ++j) {
-                if (j < L_row) {
-                    const int sb = j % S_BUFS, st = j & 1;
-                    if (j >= S_BUFS && !(ok = mbar_wait(bar(B_S_FREE + sb), ((j / S_BUFS) - 1) & 1, wc, SITE_S_FREE)))
-                        break;
-                    if (!(ok = mbar_wait(bar(B_K_FULL + st), (j >> 1) & 1, wc, SITE_K_FULL)))
+            for (int hh = 0; ok && hh <= n_half; ++hh) {
+                if (hh < n_half) {
+                    // S_hh into buffer hh % 2; its previous occupant's P V
+                    // (half-tile hh - 2) was issued in the previous iteration.
+                    const int ks = hh % L::KS;
+                    if (!(ok = mbar_wait(bar(B_K_FULL + ks), (hh / L::KS) & 1, wc, SITE_K_FULL)))
                         break;
                     tc_fence_after();
-                    const uint32_t kbase = sK + st * L::TILE_BYTES;
+                    const uint32_t kbase = sK + ks * L::H_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
-                        mma_ss(tmem + sb * TILE, smem_desc_sw128(sQ + off, 16, 1024),
-                               smem_desc_sw128(kbase + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                        mma_ss(tmem + s_col_of(hh & 1),
+                               smem_desc_sw128(sQ + (kk >> 2) * L::Q_CHUNK_BYTES + (kk & 3) * 32, 16, 1024),
+                               smem_desc_sw128(kbase + (kk >> 2) * L::H_CHUNK_BYTES + (kk & 3) * 32, 16, 1024),
+                               idesc_s, kk > 0 ? 1u : 0u);
                     }
-                    mma_commit(bar(B_S_FULL + sb));
-                    mma_commit(bar(B_K_EMPTY + st));
+                    mma_commit(bar(B_S_FULL + (hh & 1)));
+                    mma_commit(bar(B_K_EMPTY + ks));
                 }
-                if (j >= 1) {
-                    const int i = j - 1, sb = i % S_BUFS, st = i & 1;
-                    if (!(ok = mbar_wait(bar(B_P_FULL + sb), (i / S_BUFS) & 1, wc, SITE_P_FULL)))
-                        break;
-                    if (!(ok = mbar_wait(bar(B_V_FULL + st), (i >> 1) & 1, wc, SITE_V_FULL)))
+                if (hh >= 1) {
+                    const int j = hh - 1, vs = j % L::VS, buf = j & 1;
+                    if (!(ok = mbar_wait(bar(B_P_FULL + buf), (j >> 1) & 1, wc, SITE_P_FULL)) ||
+                        !(ok = mbar_wait(bar(B_V_FULL + vs), (j / L::VS) & 1, wc, SITE_V_FULL)))
                         break;
                     tc_fence_after();
-                    const uint32_t vbase = sV + st * L::TILE_BYTES;
+                    const uint32_t vbase = sV + vs * L::H_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < TILE / 16; ++kk)
-                        mma_ts(tmem + O_COL, tmem + sb * TILE + kk * 8,
-                               smem_desc_sw128(vbase + kk * 2048, L::CHUNK_BYTES, 1024), idesc_pv,
-                               (i > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < HALF / 16; ++kk)
+                        mma_ts(tmem + O_COL, tmem + s_col_of(buf) + kk * 8,
+                               smem_desc_sw128(vbase + kk * 2048, L::H_CHUNK_BYTES, 1024), idesc_pv,
+                               (j > 0 || kk > 0) ? 1u : 0u);
                     if (SPLIT_P) {
 #pragma unroll
-                        for (int kk = 0; kk < TILE / 16; ++kk)
-                            mma_ts(tmem + O_COL, tmem + sb * TILE + 64 + kk * 8,
-                                   smem_desc_sw128(vbase + kk * 2048, L::CHUNK_BYTES, 1024), idesc_pv, 1u);
+                        for (int kk = 0; kk < HALF / 16; ++kk)
+                            mma_ts(tmem + O_COL, tmem + s_col_of(buf) + HALF / 2 + kk * 8,
+                                   smem_desc_sw128(vbase + kk * 2048, L::H_CHUNK_BYTES, 1024), idesc_pv, 1u);
                     }
-                    mma_commit(bar(B_V_EMPTY + st));
-                    mma_commit(bar(B_S_FREE + sb));
+                    mma_commit(bar(B_V_EMPTY + vs));
                     mma_commit(bar(B_PV_DONE));
                 }
             }
@@ -263,7 +386,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             drain_wait(bar(B_O_FINAL), 0, p.timeout_ns);
         }
     } else {
-        // ------------------------------------------------------------- softmax
+        // ----------------------------------------------------------------- softmax
         const int t = threadIdx.x;  // == TMEM lane == query row in the tile
         const int row = qb * TILE + t;
         const bool row_valid = row < n;
@@ -272,61 +395,103 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool tail = (n % TILE) != 0;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
-        for (int i = 0; i < L_row; ++i) {
-            const int sb = i % S_BUFS;
-            const int kb = p.col_idx[row_start + i];
-            const bool partial = p.flag[row_start + i] != RA_TILE_FULL;
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_S_FULL + sb), (i / S_BUFS) & 1, wc, SITE_S_FULL));
+        uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
+        bool masked = false;
+        // CSR entry of the next tile, loaded one tile ahead of its use.
+        int next_kb = L_row > 0 ? p.col_idx[row_start] : 0;
+        int next_flag = L_row > 0 ? p.flag[row_start] : 0;
+        for (int hh = 0; hh < n_half; ++hh) {
+            const int i = hh >> 1, half = hh & 1, buf = hh & 1;
+            const uint32_t s_col = s_col_of(buf);
+            if (half == 0) {
+                // Mask of the whole tile: token-exact partial tiles use the
+                // family's element mask; the tail key tile masks keys >= n.
+                const int kb = next_kb;
+                const bool use_family = p.mode == RA_MODE_TOKEN_EXACT && next_flag != RA_TILE_FULL;
+                if (i + 1 < L_row) {
+                    next_kb = p.col_idx[row_start + i + 1];
+                    next_flag = p.flag[row_start + i + 1];
+                }
+                masked = use_family || (tail && kb == p.nb - 1);
+                if (masked) {
+                    if (use_family && row_valid) {
+                        row_keep_mask(p.g, qi, qk, kb * TILE, mk[0], mk[1], mk[2], mk[3]);
+                    } else {
+                        const int valid_cols = min(TILE, n - kb * TILE);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int v = valid_cols - 32 * c;
+                            mk[c] = v >= 32 ? 0xFFFFFFFFu : (v <= 0 ? 0u : ((1u << v) - 1u));
+                        }
+                    }
+                }
+            }
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_S_FULL + buf), (hh >> 1) & 1, wc, SITE_S_FULL));
             if (!ok)
                 break;
             tc_fence_after();
-            uint32_t r[4][32];
+            uint32_t r[2][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-                tmem_ld32(lane_base + sb * TILE + c * 32, r[c]);
+            for (int c = 0; c < 2; ++c)
+                tmem_ld32(lane_base + s_col + c * 32, r[c]);
             tmem_wait_ld();
-
-            // Mask: token-exact partial tiles use the family's element mask;
-            // the tail key tile masks keys >= n in both modes.
-            const bool use_family = p.mode == RA_MODE_TOKEN_EXACT && partial;
-            if (use_family || (tail && kb == p.nb - 1)) {
-                uint32_t mk[4];
-                if (use_family && row_valid) {
-                    row_keep_mask(p.g, qi, qk, kb * TILE, mk[0], mk[1], mk[2], mk[3]);
-                } else {
-                    const int valid_cols = min(TILE, n - kb * TILE);
+            if (masked) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int v = valid_cols - 32 * c;
-                        mk[c] = v >= 32 ? 0xFFFFFFFFu : (v <= 0 ? 0u : ((1u << v) - 1u));
-                    }
-                }
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
+                for (int c = 0; c < 2; ++c) {
+                    const uint32_t w = half ? mk[2 + c] : mk[c];
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
-                        if (!((mk[c] >> e) & 1u))
+                        if (!((w >> e) & 1u))
                             r[c][e] = __float_as_uint(-INFINITY);
+                }
             }
 
-            float mx = -INFINITY;
+            // Exponentials of the half-tile against m_use, P to TMEM; with
+            // fused_max the same pass also finds the half-tile's raw maximum.
+            auto exp_pass = [&](float m_use, bool fused_max, float& mx_out) -> float {
+                float acc[RA_SUMACC];
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+                for (int a = 0; a < RA_SUMACC; ++a)
+                    acc[a] = 0.f;
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    mx = fmaxf(mx, __uint_as_float(r[c][e]));
-            const float m_tile = mx * p.scale_log2;  // scale > 0
-
-            // Raise the running max (warp-uniformly) only when it grows by > 2^8.
-            const bool grow = m_tile > m_run + RESCALE_THRESHOLD;
-            if (__any_sync(0xFFFFFFFFu, grow)) {
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t pk[16], pl[16];
+                    if (SPLIT_P || masked) {
+                        if (fused_max)
+                            exp_chunk<0, SPLIT_P, true>(r[c], p.scale_log2, -m_use, acc, mx, pk, pl);
+                        else
+                            exp_chunk<0, SPLIT_P, false>(r[c], p.scale_log2, -m_use, acc, mx, pk, pl);
+                    } else {
+                        if (fused_max)
+                            exp_chunk<EMU_PER_32, false, true>(r[c], p.scale_log2, -m_use, acc, mx, pk, pl);
+                        else
+                            exp_chunk<EMU_PER_32, false, false>(r[c], p.scale_log2, -m_use, acc, mx, pk, pl);
+                    }
+                    tmem_st16(lane_base + s_col + c * 16, pk);
+                    if (SPLIT_P)
+                        tmem_st16(lane_base + s_col + HALF / 2 + c * 16, pl);
+                }
+#pragma unroll
+                for (int w = RA_SUMACC / 2; w >= 1; w /= 2)
+#pragma unroll
+                    for (int a = 0; a < w; ++a)
+                        acc[a] += acc[a + w];
+                mx_out = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                return acc[0];
+            };
+            // Raise the running max (warp-uniformly) when the half-tile's maximum
+            // m_tile exceeds it by more than 8: rescale O and l, once the P V of
+            // the previous half-tile has completed (the ones before it have: S_hh
+            // was issued after them).
+            bool raise_ok = true;
+            auto raise_max = [&](float m_tile) {
                 const float m_new = fmaxf(m_run, m_tile);
                 const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
-                if (i > 0) {
-                    // O holds P_0..P_{i-1} V: wait for the last PV before rescaling it.
-                    ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_PV_DONE), (i - 1) & 1, wc, SITE_PV_DONE));
-                    if (!ok)
-                        break;
+                if (hh > 0) {
+                    raise_ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_PV_DONE), (hh - 1) & 1, wc, SITE_PV_DONE));
+                    if (!raise_ok)
+                        return;
                     tc_fence_after();
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
@@ -341,31 +506,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 l_run *= alpha;
                 m_run = m_new;
-            }
-            const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-            float sum = 0.f;
+            };
+            float sum, mx_raw;
+            if (__any_sync(0xFFFFFFFFu, m_run == -INFINITY)) {
+                // No reference maximum yet in this warp: the max first, then the pass.
+                float mc[RA_MAXACC];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t pk[16], pl[16];
+                for (int a = 0; a < RA_MAXACC; ++a)
+                    mc[a] = -INFINITY;
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float p0 = fast_exp2(fmaf(__uint_as_float(r[c][e]), p.scale_log2, -m_use));
-                    const float p1 = fast_exp2(fmaf(__uint_as_float(r[c][e + 1]), p.scale_log2, -m_use));
-                    sum += p0 + p1;
-                    pk[e >> 1] = pack_bf16(p0, p1);
-                    if (SPLIT_P) {
-                        const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&pk[e >> 1]);
-                        pl[e >> 1] = pack_bf16(p0 - __low2float(hi), p1 - __high2float(hi));
-                    }
+                for (int idx = 0; idx < HALF; ++idx)
+                    mc[idx % RA_MAXACC] = fmaxf(mc[idx % RA_MAXACC], __uint_as_float(r[idx / 32][idx % 32]));
+#pragma unroll
+                for (int w = RA_MAXACC / 2; w >= 1; w /= 2)
+#pragma unroll
+                    for (int a = 0; a < w; ++a)
+                        mc[a] = fmaxf(mc[a], mc[a + w]);
+                const float m_tile = mc[0] * p.scale_log2;  // scale > 0
+                if (__any_sync(0xFFFFFFFFu, m_tile > m_run + RESCALE_THRESHOLD))
+                    raise_max(m_tile);
+                sum = exp_pass(m_run == -INFINITY ? 0.f : m_run, false, mx_raw);
+            } else {
+                // One pass against the running maximum, which the half-tile's own
+                // maximum rarely exceeds by more than 8; when it does, the pass is
+                // redone after raising the maximum (its P and sum are discarded).
+                sum = exp_pass(m_run, true, mx_raw);
+                const float m_tile = mx_raw * p.scale_log2;
+                if (__any_sync(0xFFFFFFFFu, m_tile > m_run + RESCALE_THRESHOLD)) {
+                    raise_max(m_tile);
+                    sum = exp_pass(m_run, false, mx_raw);
                 }
-                tmem_st16(lane_base + sb * TILE + c * 16, pk);
-                if (SPLIT_P)
-                    tmem_st16(lane_base + sb * TILE + 64 + c * 16, pl);
             }
+            if (!(ok = raise_ok))
+                break;
             l_run += sum;
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(B_P_FULL + sb));
+            mbar_arrive(bar(B_P_FULL + buf));
         }
 
         // ------------------------------------------------------------ epilogue
@@ -448,14 +625,14 @@ EncodeTiledFn encode_fn()
 
 // [B*H, n, d] bf16, boxes of 128 rows x 64 columns, 128-byte swizzle; rows
 // beyond n read as zero.
-ra_status make_map(CUtensorMap* map, const void* base, int BH, int n, int d)
+ra_status make_map(CUtensorMap* map, const void* base, int BH, int n, int d, int box_rows)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn)
         return fail(RA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(BH)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(n) * d * 2};
-    cuuint32_t box[3] = {64, TILE, 1};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -474,6 +651,9 @@ ra_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
     std::call_once(attr_once, [] {
         attr_err = cudaFuncSetAttribute(attn_fwd_kernel<D, SPLIT_P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         Layout<D>::SMEM_BYTES);
+        if (attr_err == cudaSuccess)  // two CTAs per SM need the whole carveout as shared memory
+            attr_err = cudaFuncSetAttribute(attn_fwd_kernel<D, SPLIT_P>,
+                                            cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     });
     if (attr_err != cudaSuccess)
         return cuda_fail(attr_err, "cudaFuncSetAttribute(attn_fwd_kernel)");
@@ -532,8 +712,8 @@ extern "C" ra_status ra_attention_fwd(const void* Q, const void* K, const void* 
         return fail(RA_ERR_INVALID_ARG, "mask has no kept tile");
     CUtensorMap mq, mk, mv;
     const int BH = B * H, n = m->geom.n;
-    if ((st = make_map(&mq, Q, BH, n, d)) != RA_OK || (st = make_map(&mk, K, BH, n, d)) != RA_OK ||
-        (st = make_map(&mv, V, BH, n, d)) != RA_OK)
+    if ((st = make_map(&mq, Q, BH, n, d, TILE)) != RA_OK || (st = make_map(&mk, K, BH, n, d, HALF)) != RA_OK ||
+        (st = make_map(&mv, V, BH, n, d, HALF)) != RA_OK)
         return st;
     FwdParams p;
     std::memset(&p, 0, sizeof p);
