@@ -61,6 +61,8 @@ def workload_desc(name, mask, mode, c):
         extra = f", r_t={mask['r_t']}, r_s={mask['r_s']}"
     if mask["family"] == "swc":
         extra = f", W={mask['window_frames']}"
+    if mask.get("sink_tokens"):
+        extra += f", {mask['sink_tokens']} global (sink) tokens"
     return (f"{name}: {mask['family']} mask{extra}, {mode} mode, f={c['f']}, s={c['s']} "
             f"({c['grid'][0]}x{c['grid'][1]}), n={c['f'] * c['s']}, B={c['B']}, H={c['H']}, d={c['d']}, "
             f"bf16 Q,K,V iid N(0,1)")

@@ -79,6 +79,10 @@ typedef struct {
     int grid_h, grid_w; /* WINDOW3D: s == grid_h * grid_w */
     int r_t, r_s;       /* WINDOW3D: temporal and spatial radius, >= 0 */
     int window_frames;  /* SWC: W >= 1 */
+    int sink_tokens;    /* every family: the first sink_tokens tokens are global --
+                           visible to every query and seeing every key ("centre band
+                           + sink" of the Radial Attention bound, sec. 4; global
+                           tokens of the tutorial, sec. 6.1).  0 (default) = none. */
 } ra_mask_params;
 
 typedef struct ra_mask ra_mask; /* opaque; owns its device arrays */

@@ -44,7 +44,7 @@ _IN_DTYPES = {np.dtype(np.uint16): 0, np.dtype(np.float32): 1, np.dtype(np.float
 class _Spec(ctypes.Structure):
     _fields_ = [("family", ctypes.c_int), ("f", ctypes.c_int), ("s", ctypes.c_int),
                 ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int), ("r_t", ctypes.c_int),
-                ("r_s", ctypes.c_int), ("window_frames", ctypes.c_int)]
+                ("r_s", ctypes.c_int), ("window_frames", ctypes.c_int), ("sink_tokens", ctypes.c_int)]
 
 
 @dataclass(frozen=True)
@@ -57,6 +57,7 @@ class MaskSpec:
     r_t: int = 0
     r_s: int = 0
     window_frames: int = 0
+    sink_tokens: int = 0
 
     @property
     def n(self) -> int:
@@ -68,7 +69,7 @@ class MaskSpec:
 
     def c(self) -> _Spec:
         return _Spec(self.family, self.f, self.s, self.grid_h, self.grid_w, self.r_t, self.r_s,
-                     self.window_frames)
+                     self.window_frames, self.sink_tokens)
 
 
 def spec_from(mask: dict, f: int, s: int, grid=(0, 0)) -> MaskSpec:
@@ -76,7 +77,7 @@ def spec_from(mask: dict, f: int, s: int, grid=(0, 0)) -> MaskSpec:
     fam = _FAMILIES[mask["family"]]
     gh, gw = grid if fam == WINDOW3D else (0, 0)
     return MaskSpec(fam, f, s, gh, gw, mask.get("r_t", 0), mask.get("r_s", 0),
-                    mask.get("window_frames", 0))
+                    mask.get("window_frames", 0), mask.get("sink_tokens", 0))
 
 
 def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:

@@ -73,6 +73,7 @@ typedef struct {
     int r_t;           /* 3D window: temporal radius */
     int r_s;           /* 3D window: spatial radius */
     int window_frames; /* sliding window: W */
+    int sink_tokens;   /* global tokens: the first sink_tokens tokens */
 } or_spec;
 
 /* Threads the parallel loops below use. */
@@ -129,10 +130,14 @@ static int or_swc_kept(const or_spec* sp, long long q, long long key)
     return (i - j) >= 0 && (i - j) <= (long long)sp->window_frames - 1;
 }
 
-/* M[q, key] == 0 ?  (token index = frame * s + position, [RA] eq. 3) */
+/* M[q, key] == 0 ?  (token index = frame * s + position, [RA] eq. 3)
+ * Global (sink) tokens -- the "sink" of the [RA] sec. 4 bound, the global
+ * tokens of [TR] sec. 6.1 -- are kept in every row and every column. */
 int oracle_kept(const or_spec* sp, long long q, long long key)
 {
     long long s = sp->s;
+    if (q < sp->sink_tokens || key < sp->sink_tokens)
+        return 1;
     switch (sp->family) {
     case OR_DENSE:
         return 1;

@@ -37,7 +37,7 @@ MODES = {"token_exact": RA_MODE_TOKEN_EXACT, "block": RA_MODE_BLOCK}
 
 class ra_mask_params(ctypes.Structure):
     _fields_ = [("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int), ("r_t", ctypes.c_int), ("r_s", ctypes.c_int),
-                ("window_frames", ctypes.c_int)]
+                ("window_frames", ctypes.c_int), ("sink_tokens", ctypes.c_int)]
 
 
 class ra_mask_info_t(ctypes.Structure):
@@ -100,9 +100,9 @@ class Mask:
     """A block-CSR mask built on the current CUDA device (owns the C handle)."""
 
     def __init__(self, family, f: int, s: int, grid_h: int = 0, grid_w: int = 0, r_t: int = 0, r_s: int = 0,
-                 window_frames: int = 0, stream=None):
+                 window_frames: int = 0, sink_tokens: int = 0, stream=None):
         fam = FAMILIES[family] if isinstance(family, str) else int(family)
-        params = ra_mask_params(grid_h, grid_w, r_t, r_s, window_frames)
+        params = ra_mask_params(grid_h, grid_w, r_t, r_s, window_frames, sink_tokens)
         handle = _MaskP()
         check(ra_build_mask(fam, f, s, ctypes.byref(params), _stream_handle(stream), ctypes.byref(handle)),
               "ra_build_mask")
@@ -145,9 +145,9 @@ class Mask:
 
 
 def build_mask(mask: dict, f: int, s: int, grid=(0, 0), stream=None) -> Mask:
-    """Mask from a dict {family, r_t, r_s, window_frames} (grid used by window3d)."""
+    """Mask from a dict {family, r_t, r_s, window_frames, sink_tokens} (grid used by window3d)."""
     return Mask(mask["family"], f, s, grid[0], grid[1], mask.get("r_t", 0), mask.get("r_s", 0),
-                mask.get("window_frames", 0), stream=stream)
+                mask.get("window_frames", 0), mask.get("sink_tokens", 0), stream=stream)
 
 
 # --------------------------------------------------------------- attention

@@ -252,6 +252,11 @@ ra_status validate_geometry(int family, int f, int s, const ra_mask_params* p, M
             return fail(RA_ERR_INVALID_ARG, "SWC needs window_frames >= 1");
         g->window_frames = p->window_frames;
     }
+    if (p) {
+        if (p->sink_tokens < 0 || p->sink_tokens > g->n)
+            return fail(RA_ERR_INVALID_ARG, "sink_tokens must be in [0, n] (got %d)", p->sink_tokens);
+        g->sink = p->sink_tokens;
+    }
     return RA_OK;
 }
 

@@ -23,13 +23,14 @@ struct MaskGeom {
     int f, s, n;  // frames, tokens per frame, n = f * s
     int grid_h, grid_w, r_t, r_s;
     int window_frames;
+    int sink;  // tokens [0, sink) are global: kept in every row and every column
 };
 
-// Calls emit(a, b) for every maximal run [a, b] of kept keys of query row
-// (frame qi, position qk) inside the key columns [c0, c1] (0 <= c0 <= c1 < n).
-// Runs are emitted in ascending order and never overlap.
+// The family's own runs (no global tokens): calls emit(a, b) for every maximal
+// run [a, b] of kept keys of query row (frame qi, position qk) inside the key
+// columns [c0, c1] (0 <= c0 <= c1 < n), in ascending order, never overlapping.
 template <class Emit>
-__device__ __forceinline__ void for_each_kept_run(const MaskGeom& g, int qi, int qk, int c0, int c1, Emit&& emit)
+__device__ __forceinline__ void for_each_family_run(const MaskGeom& g, int qi, int qk, int c0, int c1, Emit&& emit)
 {
     const int s = g.s;
     const int j0 = c0 / s, j1 = c1 / s;
@@ -92,6 +93,29 @@ __device__ __forceinline__ void for_each_kept_run(const MaskGeom& g, int qi, int
     default:
         return;
     }
+}
+
+// Calls emit(a, b) for every maximal run [a, b] of kept keys of query row
+// (frame qi, position qk) inside the key columns [c0, c1] (0 <= c0 <= c1 < n),
+// in ascending order, never overlapping.  Global (sink) tokens first: a sink
+// query keeps every key; other queries keep the sink keys and then the
+// family's keys beyond them.
+template <class Emit>
+__device__ __forceinline__ void for_each_kept_run(const MaskGeom& g, int qi, int qk, int c0, int c1, Emit&& emit)
+{
+    if (g.sink > 0) {
+        if (qi * g.s + qk < g.sink) {
+            emit(c0, c1);
+            return;
+        }
+        if (c0 < g.sink) {
+            emit(c0, min(c1, g.sink - 1));
+            c0 = g.sink;
+            if (c0 > c1)
+                return;
+        }
+    }
+    for_each_family_run(g, qi, qk, c0, c1, emit);
 }
 
 // Number of kept keys of a query row inside [c0, c1].

@@ -29,7 +29,8 @@ GAMMA = 0x9E3779B97F4A7C15
 # Workloads.  Shapes and mask parameters of the five benchmark configurations
 # (token index = frame * s + position, position = h * grid_w + w).
 # A mask entry is a dict: family in {"dense", "radial", "window3d", "swc"} plus
-# r_t / r_s (window3d) or window_frames (swc).
+# r_t / r_s (window3d) or window_frames (swc), and optionally sink_tokens
+# (global tokens; 3600 = the first frame of the 108k workload).
 # ---------------------------------------------------------------------------
 CONFIGS = {
     "tiny_radial": dict(index=0, f=8, s=64, grid=(8, 8), B=1, H=1, d=64,
@@ -40,7 +41,8 @@ CONFIGS = {
     "wan_radial": dict(index=2, f=41, s=1560, grid=(30, 52), B=1, H=40, d=128,
                        masks=[dict(family="radial"), dict(family="swc", window_frames=16)]),
     "hunyuan108k": dict(index=3, f=30, s=3600, grid=(45, 80), B=1, H=24, d=128,
-                        masks=[dict(family="radial"), dict(family="dense")]),
+                        masks=[dict(family="radial"), dict(family="dense"),
+                               dict(family="radial", sink_tokens=3600)]),
     "long460k": dict(index=4, f=128, s=3600, grid=(45, 80), B=1, H=24, d=128,
                      masks=[dict(family="radial")]),
 }

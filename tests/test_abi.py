@@ -58,6 +58,8 @@ def _build(ra, fam, f, s, params=None):
     (2, 4, 12, (3, 4, -1, 1, 0), 1),            # negative radius
     (3, 4, 12, (0, 0, 0, 0, 0), 1),             # window_frames < 1
     (1, 1 << 20, 1 << 12, None, 2),             # n beyond the builder's limit
+    (1, 4, 4, (0, 0, 0, 0, 0, -1), 1),          # negative sink_tokens
+    (1, 4, 4, (0, 0, 0, 0, 0, 17), 1),          # sink_tokens > n
 ])
 def test_build_mask_rejects_bad_arguments(ra, fam, f, s, params, status):
     p = ra.ra_mask_params(*params) if params else None

@@ -22,7 +22,8 @@ MODES = {"token_exact": oracle.TOKEN_EXACT, "block": oracle.BLOCK}
 def _run(spec: oracle.MaskSpec, Qh, Kh, Vh, mode: str, lse=False):
     ra = _gpu.ra()
     fam = {oracle.DENSE: "dense", oracle.RADIAL: "radial", oracle.WINDOW3D: "window3d", oracle.SWC: "swc"}[spec.family]
-    m = ra.Mask(fam, spec.f, spec.s, spec.grid_h, spec.grid_w, spec.r_t, spec.r_s, spec.window_frames)
+    m = ra.Mask(fam, spec.f, spec.s, spec.grid_h, spec.grid_w, spec.r_t, spec.r_s, spec.window_frames,
+                spec.sink_tokens)
     q, k, v = (_gpu.to_device(t) for t in (Qh, Kh, Vh))
     B, H, n, d = q.shape
     out_lse = torch.empty((B, H, n), dtype=torch.float32, device="cuda") if lse else None
@@ -92,6 +93,8 @@ EDGE_CASES = [
     (oracle.MaskSpec(oracle.WINDOW3D, 5, 99, 9, 11, 2, 4), 2, 1, 128),
     (oracle.MaskSpec(oracle.DENSE, 3, 77), 1, 1, 64),
     (oracle.MaskSpec(oracle.RADIAL, 64, 16), 1, 1, 128),   # sub-sampled diagonals (w > s)
+    (oracle.MaskSpec(oracle.RADIAL, 11, 100, sink_tokens=100), 1, 2, 128),   # first frame global
+    (oracle.MaskSpec(oracle.SWC, 9, 130, window_frames=2, sink_tokens=200), 1, 1, 64),
 ]
 
 
@@ -169,7 +172,8 @@ def test_bounded_wait_selftest_reports_timeout():
 # ------------------------------------------------- full-size configs (sampled)
 
 FULL = [("wan_radial", 0, "block"), ("wan_radial", 1, "block"), ("hunyuan108k", 0, "block"),
-        ("hunyuan108k", 1, "block"), ("long460k", 0, "block"), ("hunyuan108k", 0, "token_exact")]
+        ("hunyuan108k", 1, "block"), ("long460k", 0, "block"), ("hunyuan108k", 0, "token_exact"),
+        ("hunyuan108k", 2, "block"), ("hunyuan108k", 2, "token_exact")]
 
 
 @pytest.mark.parametrize("name,mask_i,mode", FULL, ids=lambda x: str(x))

@@ -12,7 +12,8 @@ pytestmark = pytest.mark.gpu
 def _gpu_mask(spec: oracle.MaskSpec):
     ra = _gpu.ra()
     fam = {oracle.DENSE: "dense", oracle.RADIAL: "radial", oracle.WINDOW3D: "window3d", oracle.SWC: "swc"}[spec.family]
-    return ra.Mask(fam, spec.f, spec.s, spec.grid_h, spec.grid_w, spec.r_t, spec.r_s, spec.window_frames)
+    return ra.Mask(fam, spec.f, spec.s, spec.grid_h, spec.grid_w, spec.r_t, spec.r_s, spec.window_frames,
+                   spec.sink_tokens)
 
 
 def _assert_csr_equal(got: dict, want: dict):
@@ -47,6 +48,10 @@ def _random_specs():
             specs.append(oracle.MaskSpec(fam, f, int(rng.integers(1, 300)), window_frames=int(rng.integers(1, 20))))
         else:
             specs.append(oracle.MaskSpec(fam, f, int(rng.integers(1, 300))))
+    # global (sink) tokens on top of each family, including a sink longer than a tile
+    for k, sp in enumerate(list(specs[:12])):
+        specs.append(oracle.MaskSpec(sp.family, sp.f, sp.s, sp.grid_h, sp.grid_w, sp.r_t, sp.r_s,
+                                     sp.window_frames, sink_tokens=min(sp.n, [1, 37, 128, 300][k % 4])))
     return specs
 
 

@@ -35,6 +35,7 @@ MUTANTS = {
     "value_of_query_row": ("or_load(V, dtype, kvbase + idx[t] * d + c)", "or_load(V, dtype, kvbase + q * d + c)"),
     "block_tile_of_query": ("[(long long)row_tile_slot[r] * nb + key / OR_TILE]", "[(long long)row_tile_slot[r] * nb + q / OR_TILE]"),
     "lse_without_max": ("lse[r] = mx + log(denom);", "lse[r] = log(denom);"),
+    "sink_only_keys": ("if (q < sp->sink_tokens || key < sp->sink_tokens)", "if (key < sp->sink_tokens)"),
 }
 
 
@@ -58,6 +59,11 @@ def _pins_hold(orc) -> bool:
         return False
     if not np.array_equal(orc.dense_mask(MaskSpec(SWC, 6, 5, window_frames=2)).astype(bool),
                           _pins.swc_mask_frames(6, 5, 2)):
+        return False
+    sink_want = _pins.radial_mask_literal(7, 9)
+    sink_want[:10, :] = True
+    sink_want[:, :10] = True
+    if not np.array_equal(orc.dense_mask(MaskSpec(RADIAL, 7, 9, sink_tokens=10)).astype(bool), sink_want):
         return False
     spec = MaskSpec(RADIAL, 11, 100)
     lit = _pins.radial_mask_literal(11, 100)

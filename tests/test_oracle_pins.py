@@ -103,6 +103,19 @@ def test_dense_family_keeps_everything(orc):
     assert orc.dense_mask(MaskSpec(DENSE, 3, 5)).all()
 
 
+@pytest.mark.parametrize("base,sink", [
+    (MaskSpec(RADIAL, 9, 20), 1), (MaskSpec(RADIAL, 12, 7), 20), (MaskSpec(SWC, 8, 11, window_frames=2), 11),
+    (MaskSpec(WINDOW3D, 4, 12, 3, 4, 1, 1), 5), (MaskSpec(RADIAL, 5, 9), 45)])
+def test_sink_tokens_are_global(orc, base, sink):
+    """Global tokens: kept in every row and every column, on top of the family."""
+    import dataclasses
+    spec = dataclasses.replace(base, sink_tokens=sink)
+    want = _literal_mask(base).copy()
+    want[:sink, :] = True
+    want[:, :sink] = True
+    assert np.array_equal(orc.dense_mask(spec).astype(bool), want)
+
+
 # ------------------------------------------------------------------ tiles/CSR
 
 def _literal_mask(spec: MaskSpec) -> np.ndarray:
