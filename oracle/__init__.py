@@ -109,6 +109,9 @@ def load_library(path: str):
     lib.oracle_attention_rows.argtypes = [vp, vp, vp, c_int, i64, c_int, P, c_int, ctypes.c_double, i64,
                                           vp, vp, vp, vp, vp, vp, vp]
     lib.oracle_attention_rows.restype = None
+    lib.oracle_attention_bwd.argtypes = [vp, vp, vp, vp, c_int, i64, c_int, P, c_int, ctypes.c_double, vp, vp, vp,
+                                         vp]
+    lib.oracle_attention_bwd.restype = None
     return lib
 
 
@@ -196,6 +199,27 @@ class Oracle:
                                        row_q.ctypes.data, tile_flags.ctypes.data, slot.ctypes.data,
                                        O.ctypes.data, lse.ctypes.data, nkeys.ctypes.data)
         return O, lse, nkeys
+
+    def attention_bwd(self, Q, K, V, dO, spec: MaskSpec, mode: int, scale: float):
+        """fp64 gradients dQ, dK, dV of the masked attention for every (b, h) slice.
+
+        Q, K, V, dO: [B, H, n, d] arrays (bf16 bit patterns, float32 or float64).
+        Returns three float64 arrays of the same shape.  O(B H n^2 d): small n only."""
+        Q, K, V, dO = (np.ascontiguousarray(t) for t in (Q, K, V, dO))
+        assert Q.dtype == K.dtype == V.dtype == dO.dtype and Q.dtype in _IN_DTYPES
+        B, H, n, d = Q.shape
+        assert n == spec.n
+        flags = (self.tile_counts(spec) > 0).astype(np.uint8) if mode == BLOCK else np.zeros(1, np.uint8)
+        out = [np.empty((B, H, n, d), dtype=np.float64) for _ in range(3)]
+        sp = spec.c()
+        for b in range(B):
+            for h in range(H):
+                self.lib.oracle_attention_bwd(Q[b, h].ctypes.data, K[b, h].ctypes.data, V[b, h].ctypes.data,
+                                              dO[b, h].ctypes.data, _IN_DTYPES[Q.dtype], n, d, ctypes.byref(sp), mode,
+                                              float(scale), flags.ctypes.data, out[0][b, h].ctypes.data,
+                                              out[1][b, h].ctypes.data, out[2][b, h].ctypes.data)
+        return tuple(out)
+
 
 
 def default() -> Oracle:

@@ -300,3 +300,82 @@ void oracle_attention_rows(const void* Q, const void* K, const void* V, int dtyp
         free(acc);
     }
 }
+
+/*
+ * Gradients of the masked softmax attention ([RA] eq. 2) for one (batch, head)
+ * slice, by the chain rule written out in its plainest order:
+ *   x_ij  = scale <Q_i, K_j>,  P_ij = exp(x_ij - lse_i) over the row's keys
+ *   O_i   = sum_j P_ij V_j,    D_i  = <dO_i, O_i>
+ *   dP_ij = <dO_i, V_j>,       dS_ij = P_ij (dP_ij - D_i)
+ *   dQ_i  = scale sum_j dS_ij K_j
+ *   dK_j  = scale sum_i dS_ij Q_i
+ *   dV_j  = sum_i P_ij dO_i
+ * Keys of row i as in oracle_attention_rows (token-exact: kept pairs; block:
+ * every valid key of a kept tile, from tile_flags[qb * nb + kb]).
+ * Q, K, V, dO: [n, d] (dtype as in oracle_attention_rows); dQ, dK, dV: [n, d]
+ * fp64, overwritten.  O(n^2 d): small n only.
+ */
+void oracle_attention_bwd(const void* Q, const void* K, const void* V, const void* dO, int dtype, long long n,
+                          int d, const or_spec* sp, int mode, double scale, const unsigned char* tile_flags,
+                          double* dQ, double* dK, double* dV)
+{
+    long long nb = (n + OR_TILE - 1) / OR_TILE;
+    double* x = (double*)malloc(sizeof(double) * (size_t)n);
+    unsigned char* use = (unsigned char*)malloc((size_t)n);
+    double* o = (double*)malloc(sizeof(double) * (size_t)d);
+    for (long long t = 0; t < n * d; t++)
+        dQ[t] = dK[t] = dV[t] = 0.0;
+    for (long long i = 0; i < n; i++) {
+        double mx = -INFINITY;
+        for (long long j = 0; j < n; j++) {
+            if (mode == OR_TOKEN_EXACT)
+                use[j] = (unsigned char)oracle_kept(sp, i, j);
+            else
+                use[j] = tile_flags[(i / OR_TILE) * nb + j / OR_TILE] != 0;
+            if (!use[j])
+                continue;
+            double dot = 0.0;
+            for (int c = 0; c < d; c++)
+                dot += or_load(Q, dtype, i * d + c) * or_load(K, dtype, j * d + c);
+            x[j] = scale * dot;
+            if (x[j] > mx)
+                mx = x[j];
+        }
+        if (mx == -INFINITY)
+            continue; /* a row with no key: no gradient */
+        double denom = 0.0;
+        for (long long j = 0; j < n; j++)
+            if (use[j])
+                denom += exp(x[j] - mx);
+        double lse = mx + log(denom);
+        /* O_i and D_i */
+        for (int c = 0; c < d; c++)
+            o[c] = 0.0;
+        for (long long j = 0; j < n; j++)
+            if (use[j]) {
+                double pij = exp(x[j] - lse);
+                for (int c = 0; c < d; c++)
+                    o[c] += pij * or_load(V, dtype, j * d + c);
+            }
+        double Di = 0.0;
+        for (int c = 0; c < d; c++)
+            Di += or_load(dO, dtype, i * d + c) * o[c];
+        for (long long j = 0; j < n; j++) {
+            if (!use[j])
+                continue;
+            double pij = exp(x[j] - lse);
+            double dpij = 0.0;
+            for (int c = 0; c < d; c++)
+                dpij += or_load(dO, dtype, i * d + c) * or_load(V, dtype, j * d + c);
+            double dsij = pij * (dpij - Di);
+            for (int c = 0; c < d; c++) {
+                dQ[i * d + c] += scale * dsij * or_load(K, dtype, j * d + c);
+                dK[j * d + c] += scale * dsij * or_load(Q, dtype, i * d + c);
+                dV[j * d + c] += pij * or_load(dO, dtype, i * d + c);
+            }
+        }
+    }
+    free(x);
+    free(use);
+    free(o);
+}

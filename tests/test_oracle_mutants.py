@@ -36,6 +36,11 @@ MUTANTS = {
     "block_tile_of_query": ("[(long long)row_tile_slot[r] * nb + key / OR_TILE]", "[(long long)row_tile_slot[r] * nb + q / OR_TILE]"),
     "lse_without_max": ("lse[r] = mx + log(denom);", "lse[r] = log(denom);"),
     "sink_only_keys": ("if (q < sp->sink_tokens || key < sp->sink_tokens)", "if (key < sp->sink_tokens)"),
+    "bwd_dropped_D": ("double dsij = pij * (dpij - Di);", "double dsij = pij * dpij;"),
+    "bwd_dK_from_K": ("dK[j * d + c] += scale * dsij * or_load(Q, dtype, i * d + c);",
+                      "dK[j * d + c] += scale * dsij * or_load(K, dtype, i * d + c);"),
+    "bwd_dV_unweighted": ("dV[j * d + c] += pij * or_load(dO, dtype, i * d + c);",
+                          "dV[j * d + c] += or_load(dO, dtype, i * d + c);"),
 }
 
 
@@ -89,6 +94,17 @@ def _pins_hold(orc) -> bool:
             want_lse = torch.logsumexp(t(sc).masked_fill(~t(mask), -math.inf), dim=-1).numpy()[rows]
             if not (np.allclose(O, want, atol=1e-12, rtol=0) and np.allclose(lse, want_lse, atol=1e-12, rtol=0)):
                 return False
+    # backward against autograd on a small radial case
+    bspec = MaskSpec(RADIAL, 6, 10)
+    blit = _pins.radial_mask_literal(6, 10)
+    Q, K, V, dO = (rng.standard_normal((1, 1, bspec.n, 8)) for _ in range(4))
+    got = orc.attention_bwd(Q, K, V, dO, bspec, TOKEN_EXACT, 0.3)
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (Q, K, V))
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=torch.from_numpy(blit), scale=0.3)
+    out.backward(torch.from_numpy(dO))
+    for g, w in zip(got, (tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy())):
+        if not np.allclose(g, w, atol=1e-10, rtol=0):
+            return False
     return True
 
 
