@@ -112,6 +112,12 @@ def load_library(path: str):
     lib.oracle_attention_bwd.argtypes = [vp, vp, vp, vp, c_int, i64, c_int, P, c_int, ctypes.c_double, vp, vp, vp,
                                          vp]
     lib.oracle_attention_bwd.restype = None
+    lib.oracle_attention_bwd_query_rows.argtypes = [vp, vp, vp, vp, c_int, i64, c_int, P, c_int, ctypes.c_double,
+                                                    i64, vp, vp, vp, vp, vp]
+    lib.oracle_attention_bwd_query_rows.restype = None
+    lib.oracle_attention_bwd_key_rows.argtypes = [vp, vp, vp, vp, c_int, i64, c_int, P, c_int, ctypes.c_double,
+                                                  vp, i64, vp, vp, vp]
+    lib.oracle_attention_bwd_key_rows.restype = None
     return lib
 
 
@@ -220,6 +226,51 @@ class Oracle:
                                               out[1][b, h].ctypes.data, out[2][b, h].ctypes.data)
         return tuple(out)
 
+
+    def attention_bwd_query_rows(self, Q, K, V, dO, spec: MaskSpec, mode: int, scale: float, row_bh, row_q):
+        """fp64 dQ of the listed query rows (b*H + h, q); [rows, d].  O(keys * d) per row."""
+        Q, K, V, dO = (np.ascontiguousarray(t) for t in (Q, K, V, dO))
+        assert Q.dtype == K.dtype == V.dtype == dO.dtype and Q.dtype in _IN_DTYPES
+        n, d = Q.shape[-2], Q.shape[-1]
+        assert n == spec.n
+        row_bh = np.ascontiguousarray(row_bh, dtype=np.int64)
+        row_q = np.ascontiguousarray(row_q, dtype=np.int64)
+        nrows = len(row_q)
+        if mode == BLOCK:
+            qbs, slot = np.unique(row_q // TILE, return_inverse=True)
+            tile_flags = (self.tile_counts(spec, qbs) > 0).astype(np.uint8)
+            slot = np.ascontiguousarray(slot, dtype=np.int32)
+        else:
+            tile_flags = np.zeros(1, dtype=np.uint8)
+            slot = np.zeros(max(nrows, 1), dtype=np.int32)
+        dQ = np.empty((nrows, d), dtype=np.float64)
+        sp = spec.c()
+        self.lib.oracle_attention_bwd_query_rows(Q.ctypes.data, K.ctypes.data, V.ctypes.data, dO.ctypes.data,
+                                                 _IN_DTYPES[Q.dtype], n, d, ctypes.byref(sp), mode, float(scale),
+                                                 nrows, row_bh.ctypes.data, row_q.ctypes.data,
+                                                 tile_flags.ctypes.data, slot.ctypes.data, dQ.ctypes.data)
+        return dQ
+
+    def attention_bwd_key_rows(self, Q, K, V, dO, spec: MaskSpec, mode: int, scale: float, keys):
+        """fp64 dK, dV of the listed key rows of ONE (b, h) slice: Q, K, V, dO are
+        [n, d].  Returns ([len(keys), d], [len(keys), d]).  O(n * keys-per-row * d)."""
+        Q, K, V, dO = (np.ascontiguousarray(t) for t in (Q, K, V, dO))
+        assert Q.dtype == K.dtype == V.dtype == dO.dtype and Q.dtype in _IN_DTYPES and Q.ndim == 2
+        n, d = Q.shape
+        assert n == spec.n
+        keys = np.ascontiguousarray(keys, dtype=np.int64)
+        if mode == BLOCK:
+            tile_flags = np.ascontiguousarray((self.tile_counts(spec) > 0).astype(np.uint8))
+        else:
+            tile_flags = np.zeros(1, dtype=np.uint8)
+        dK = np.empty((len(keys), d), dtype=np.float64)
+        dV = np.empty((len(keys), d), dtype=np.float64)
+        sp = spec.c()
+        self.lib.oracle_attention_bwd_key_rows(Q.ctypes.data, K.ctypes.data, V.ctypes.data, dO.ctypes.data,
+                                               _IN_DTYPES[Q.dtype], n, d, ctypes.byref(sp), mode, float(scale),
+                                               tile_flags.ctypes.data, len(keys), keys.ctypes.data,
+                                               dK.ctypes.data, dV.ctypes.data)
+        return dK, dV
 
 
 def default() -> Oracle:

@@ -379,3 +379,164 @@ void oracle_attention_bwd(const void* Q, const void* K, const void* V, const voi
     free(use);
     free(o);
 }
+
+/* Keys of query q (token-exact: M[q, key] == 0; block: every key of a kept
+ * tile, flags[key / 128] != 0 with flags the query tile's row of tile flags),
+ * their scores x = scale <Q_q, K_key> and the row's log-sum-exp.  Returns the
+ * number of keys; idx / x receive them. */
+static long long or_row_scores(const void* Q, const void* K, int dtype, long long n, int d, const or_spec* sp,
+                               int mode, double scale, long long q, const unsigned char* flags,
+                               long long qoff, long long kvbase, long long* idx, double* x, double* lse)
+{
+    long long m = 0;
+    for (long long key = 0; key < n; key++) {
+        int use = mode == OR_TOKEN_EXACT ? oracle_kept(sp, q, key) : flags[key / OR_TILE] != 0;
+        if (!use)
+            continue;
+        long long koff = kvbase + key * d;
+        double dot = 0.0;
+        for (int c = 0; c < d; c++)
+            dot += or_load(Q, dtype, qoff + c) * or_load(K, dtype, koff + c);
+        x[m] = dot * scale;
+        idx[m] = key;
+        m++;
+    }
+    if (m == 0) {
+        *lse = -INFINITY;
+        return 0;
+    }
+    double mx = x[0];
+    for (long long t = 1; t < m; t++)
+        if (x[t] > mx)
+            mx = x[t];
+    double denom = 0.0;
+    for (long long t = 0; t < m; t++)
+        denom += exp(x[t] - mx);
+    *lse = mx + log(denom);
+    return m;
+}
+
+/*
+ * dQ of listed query rows, from the same definitions as oracle_attention_bwd
+ * (dQ_i = scale sum_j P_ij (<dO_i, V_j> - D_i) K_j, D_i = <dO_i, O_i>), one row
+ * at a time in O(keys * d): for sampled rows of workloads too large for the
+ * whole backward.  Rows and tile flags as in oracle_attention_rows; dQ is
+ * [nrows, d] fp64.
+ */
+void oracle_attention_bwd_query_rows(const void* Q, const void* K, const void* V, const void* dO, int dtype,
+                                     long long n, int d, const or_spec* sp, int mode, double scale, long long nrows,
+                                     const long long* row_bh, const long long* row_q,
+                                     const unsigned char* tile_flags, const int* row_tile_slot, double* dQ)
+{
+    long long nb = (n + OR_TILE - 1) / OR_TILE;
+#pragma omp parallel
+    {
+        double* x = (double*)malloc(sizeof(double) * (size_t)n);
+        long long* idx = (long long*)malloc(sizeof(long long) * (size_t)n);
+        double* o = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 4)
+        for (long long r = 0; r < nrows; r++) {
+            long long q = row_q[r];
+            long long qoff = (row_bh[r] * n + q) * d;
+            long long kvbase = row_bh[r] * n * d;
+            const unsigned char* flags = mode == OR_TOKEN_EXACT ? NULL : tile_flags + (long long)row_tile_slot[r] * nb;
+            double lse;
+            long long m = or_row_scores(Q, K, dtype, n, d, sp, mode, scale, q, flags, qoff, kvbase, idx, x, &lse);
+            for (int c = 0; c < d; c++)
+                dQ[r * d + c] = 0.0;
+            if (m == 0)
+                continue;
+            for (int c = 0; c < d; c++)
+                o[c] = 0.0;
+            for (long long t = 0; t < m; t++) {
+                long long koff = kvbase + idx[t] * d;
+                double p = exp(x[t] - lse);
+                for (int c = 0; c < d; c++)
+                    o[c] += p * or_load(V, dtype, koff + c);
+            }
+            double D = 0.0;
+            for (int c = 0; c < d; c++)
+                D += or_load(dO, dtype, qoff + c) * o[c];
+            for (long long t = 0; t < m; t++) {
+                long long koff = kvbase + idx[t] * d;
+                double p = exp(x[t] - lse), dp = 0.0;
+                for (int c = 0; c < d; c++)
+                    dp += or_load(dO, dtype, qoff + c) * or_load(V, dtype, koff + c);
+                double ds = p * (dp - D);
+                for (int c = 0; c < d; c++)
+                    dQ[r * d + c] += scale * ds * or_load(K, dtype, koff + c);
+            }
+        }
+        free(x);
+        free(idx);
+        free(o);
+    }
+}
+
+/*
+ * dK and dV of listed key rows of one (batch, head) slice (Q, K, V, dO: [n, d]):
+ * first lse_i and D_i of every query row, then for each listed key j
+ *   dK_j = scale sum_i P_ij (<dO_i, V_j> - D_i) Q_i,   dV_j = sum_i P_ij dO_i
+ * over the queries i whose row keeps j.  O(n * keys * d) for the statistics,
+ * O(n * d) per listed key.  tile_flags: the whole nb x nb table (block mode).
+ * dK, dV: [nkeys, d] fp64.
+ */
+void oracle_attention_bwd_key_rows(const void* Q, const void* K, const void* V, const void* dO, int dtype,
+                                   long long n, int d, const or_spec* sp, int mode, double scale,
+                                   const unsigned char* tile_flags, long long nkeys, const long long* key_idx,
+                                   double* dK, double* dV)
+{
+    long long nb = (n + OR_TILE - 1) / OR_TILE;
+    double* lse = (double*)malloc(sizeof(double) * (size_t)n);
+    double* Dv = (double*)malloc(sizeof(double) * (size_t)n);
+#pragma omp parallel
+    {
+        double* x = (double*)malloc(sizeof(double) * (size_t)n);
+        long long* idx = (long long*)malloc(sizeof(long long) * (size_t)n);
+        double* o = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 16)
+        for (long long i = 0; i < n; i++) {
+            const unsigned char* flags = mode == OR_TOKEN_EXACT ? NULL : tile_flags + (i / OR_TILE) * nb;
+            long long m = or_row_scores(Q, K, dtype, n, d, sp, mode, scale, i, flags, i * d, 0, idx, x, &lse[i]);
+            for (int c = 0; c < d; c++)
+                o[c] = 0.0;
+            for (long long t = 0; t < m; t++) {
+                double p = exp(x[t] - lse[i]);
+                for (int c = 0; c < d; c++)
+                    o[c] += p * or_load(V, dtype, idx[t] * d + c);
+            }
+            double D = 0.0;
+            for (int c = 0; c < d; c++)
+                D += or_load(dO, dtype, i * d + c) * o[c];
+            Dv[i] = D;
+        }
+        free(x);
+        free(idx);
+        free(o);
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long long r = 0; r < nkeys; r++) {
+        long long j = key_idx[r];
+        for (int c = 0; c < d; c++)
+            dK[r * d + c] = dV[r * d + c] = 0.0;
+        for (long long i = 0; i < n; i++) {
+            int use = mode == OR_TOKEN_EXACT ? oracle_kept(sp, i, j)
+                                             : tile_flags[(i / OR_TILE) * nb + j / OR_TILE] != 0;
+            if (!use)
+                continue;
+            double dot = 0.0, dp = 0.0;
+            for (int c = 0; c < d; c++) {
+                dot += or_load(Q, dtype, i * d + c) * or_load(K, dtype, j * d + c);
+                dp += or_load(dO, dtype, i * d + c) * or_load(V, dtype, j * d + c);
+            }
+            double p = exp(scale * dot - lse[i]);
+            double ds = p * (dp - Dv[i]);
+            for (int c = 0; c < d; c++) {
+                dK[r * d + c] += scale * ds * or_load(Q, dtype, i * d + c);
+                dV[r * d + c] += p * or_load(dO, dtype, i * d + c);
+            }
+        }
+    }
+    free(lse);
+    free(Dv);
+}

@@ -118,6 +118,19 @@ def qkv_bf16(name: str, B: int | None = None, H: int | None = None):
     return tuple(normal_bf16(seed, t, shape) for t in range(3))
 
 
+# Stream id of the output gradient dO (the forward inputs use ids 0, 1, 2 per
+# rank, so it stays clear of every rank's Q, K, V).
+DOUT_TENSOR_ID = 1 << 20
+
+
+def dout_bf16(name: str, B: int | None = None, H: int | None = None) -> np.ndarray:
+    """Output gradient dO of a named workload, i.i.d. N(0,1) bf16 bits, [B, H, n, d]."""
+    c = CONFIGS[name]
+    B = c["B"] if B is None else B
+    H = c["H"] if H is None else H
+    return normal_bf16(config_seed(name), DOUT_TENSOR_ID, (B, H, c["f"] * c["s"], c["d"]))
+
+
 def _mix(z: int) -> int:
     z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & MASK64
     z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & MASK64

@@ -41,6 +41,13 @@ MUTANTS = {
                       "dK[j * d + c] += scale * dsij * or_load(K, dtype, i * d + c);"),
     "bwd_dV_unweighted": ("dV[j * d + c] += pij * or_load(dO, dtype, i * d + c);",
                           "dV[j * d + c] += or_load(dO, dtype, i * d + c);"),
+    "rows_dropped_scale": ("x[m] = dot * scale;", "x[m] = dot;"),
+    "rows_transposed_key_operand": ("dot += or_load(Q, dtype, qoff + c) * or_load(K, dtype, koff + c);",
+                                    "dot += or_load(Q, dtype, qoff + c) * or_load(K, dtype, kvbase + c * n + key);"),
+    "qrows_dropped_D": ("double ds = p * (dp - D);", "double ds = p * dp;"),
+    "krows_dV_unweighted": ("dV[r * d + c] += p * or_load(dO, dtype, i * d + c);",
+                            "dV[r * d + c] += or_load(dO, dtype, i * d + c);"),
+    "krows_lse_of_key": ("double p = exp(scale * dot - lse[i]);", "double p = exp(scale * dot - lse[j]);"),
 }
 
 
@@ -102,8 +109,16 @@ def _pins_hold(orc) -> bool:
     tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (Q, K, V))
     out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=torch.from_numpy(blit), scale=0.3)
     out.backward(torch.from_numpy(dO))
-    for g, w in zip(got, (tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy())):
+    grads = (tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy())
+    for g, w in zip(got, grads):
         if not np.allclose(g, w, atol=1e-10, rtol=0):
+            return False
+    # the row-at-a-time dQ and key-at-a-time dK, dV on the same case
+    rows = np.array([0, 7, 31, bspec.n - 1])
+    dq = orc.attention_bwd_query_rows(Q, K, V, dO, bspec, TOKEN_EXACT, 0.3, np.zeros_like(rows), rows)
+    dk, dv = orc.attention_bwd_key_rows(Q[0, 0], K[0, 0], V[0, 0], dO[0, 0], bspec, TOKEN_EXACT, 0.3, rows)
+    for g, w in zip((dq, dk, dv), grads):
+        if not np.allclose(g, w[0, 0, rows], atol=1e-10, rtol=0):
             return False
     return True
 
