@@ -4,7 +4,10 @@
     python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
 
 One step = one ra_attention_fwd call over every batch element and head of the
-workload (mask built once beforehand: it is static).  Default workload: the
+workload (mask built once beforehand: it is static).  With --pass bwd a step is
+one ra_attention_bwd call instead (dQ, dK, dV from the forward's O and lse and a
+seeded dO), counted at 10 * d FLOP per computed pair per head (the five
+products S, dP, dQ, dK, dV; the kernels recompute S and dP in both passes).  Default workload: the
 HunyuanVideo-shaped radial configuration (f=30 frames, s=3600 tokens per
 frame, n=108000, 24 heads, d=128), eq. 4 mask at 128x128 tiles, block mode.
 
@@ -34,9 +37,15 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "radial sparse-attn fwd ms & effective TFLOP/s (bf16, % of TC peak), 1 B200"
+METRIC_BWD = "radial sparse-attn bwd ms & effective TFLOP/s (bf16, % of TC peak), 1 B200"
+METRIC_STREAM = "SWC streaming step (KV ring cache) ms per frame & effective TFLOP/s (bf16), 1 B200"
 L2_BYTES = 126 * 1024 * 1024
-ATTN_SOURCES = ["static_sparse_attention_b200/csrc/ra_attention.cu", "static_sparse_attention_b200/csrc/ra_sm100.cuh",
-                "static_sparse_attention_b200/csrc/ra_mask_math.cuh"]
+ATTN_SOURCES = {
+    "fwd": ["static_sparse_attention_b200/csrc/ra_attention.cu", "static_sparse_attention_b200/csrc/ra_sm100.cuh",
+            "static_sparse_attention_b200/csrc/ra_mask_math.cuh"],
+    "bwd": ["static_sparse_attention_b200/csrc/ra_attention_bwd.cu", "static_sparse_attention_b200/csrc/ra_sm100.cuh",
+            "static_sparse_attention_b200/csrc/ra_mask_math.cuh"],
+}
 
 
 def parse_args():
@@ -52,6 +61,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (small profiling cases)")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd", "stream"],
+                    help="time the forward (default), the backward, or the streaming SWC step")
     return ap.parse_args()
 
 
@@ -77,24 +88,25 @@ def measured_peaks():
     return 1590.0, 1400.0, 6650.0, "fallback"
 
 
-def sources_sha256():
+def sources_sha256(kind="fwd"):
     h = hashlib.sha256()
-    for rel in ATTN_SOURCES:
+    for rel in ATTN_SOURCES[kind]:
         with open(os.path.join(ROOT, rel), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload, mode, mask_family):
-    """DRAM bytes per launch of the forward kernel from the committed ncu summary,
-    if it was taken on the current kernel sources (else None)."""
-    path = os.path.join(ROOT, "profiles", "attn_fwd_traffic.txt")
+def recorded_traffic(workload, mode, mask_family, kind="fwd"):
+    """DRAM bytes per launch (per call, for the backward's kernels together) from
+    the committed ncu summary, if it was taken on the current kernel sources
+    (else None)."""
+    path = os.path.join(ROOT, "profiles", f"attn_{kind}_traffic.txt")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     key = f"{workload}/{mask_family}/{mode}"
     m = re.search(rf"^{re.escape(key)}\s+sources=(\w+)\s+dram_bytes_per_launch=(\d+)", text, flags=re.M)
-    if not m or m.group(1) != sources_sha256():
+    if not m or m.group(1) != sources_sha256(kind):
         return None
     return int(m.group(2))
 
@@ -181,15 +193,17 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
-def flops_per_call(info, c, mode):
+def flops_per_call(info, c, mode, kind="fwd"):
     pairs = info["block_pairs"] if mode == "block" else info["kept_pairs"]
-    return 4.0 * c["d"] * pairs * c["B"] * c["H"]
+    return (4.0 if kind == "fwd" else 10.0) * c["d"] * pairs * c["B"] * c["H"]
 
 
-def cpu_oracle_sample(name, mask, mode, c, target_s=15.0, seed_rank=0):
+def cpu_oracle_sample(name, mask, mode, c, target_s=15.0, seed_rank=0, kind="fwd"):
     """Time the oracle (as it stands) on a bounded sample of the workload: query
-    rows of head 0 until about target_s seconds of CPU work.  Returns
-    (TFLOP/s, threads, sample description)."""
+    rows of head 0 until about target_s seconds of CPU work.  Forward: the
+    attention of each row (4 d FLOP per computed pair).  Backward: the dQ of each
+    row, which needs its S, O, dP and dQ (8 d FLOP per computed pair).
+    Returns (TFLOP/s, threads, sample description)."""
     import oracle
     orc = oracle.default()
     spec = oracle.spec_from(mask, c["f"], c["s"], c["grid"])
@@ -197,21 +211,30 @@ def cpu_oracle_sample(name, mask, mode, c, target_s=15.0, seed_rank=0):
     shape = (1, 1, n, d)
     seed = synth.config_seed(name) + 1000 * seed_rank
     Q, K, V = (synth.normal_bf16(seed, t, shape) for t in range(3))
+    dO = synth.normal_bf16(seed, synth.DOUT_TENSOR_ID, shape) if kind == "bwd" else None
     omode = oracle.BLOCK if mode == "block" else oracle.TOKEN_EXACT
+    per_pair = 4.0 * d if kind == "fwd" else 8.0 * d
     rows_all = synth.sample_rows(seed, c["f"], c["s"], count=min(n, 4096))
     rng = np.random.default_rng(seed)
     rng.shuffle(rows_all)
     nrows, done_rows, flop, elapsed = 8, 0, 0.0, 0.0
     while elapsed < target_s and done_rows < len(rows_all):
         rows = rows_all[done_rows:done_rows + nrows]
+        zeros = np.zeros(len(rows), np.int64)
         t0 = time.perf_counter()
-        _, _, nk = orc.attention_rows(Q, K, V, spec, omode, 1 / math.sqrt(d), np.zeros(len(rows), np.int64), rows)
+        if kind == "fwd":
+            _, _, nk = orc.attention_rows(Q, K, V, spec, omode, 1 / math.sqrt(d), zeros, rows)
+        else:
+            _, nk = orc.attention_bwd_query_rows(Q, K, V, dO, spec, omode, 1 / math.sqrt(d), zeros, rows,
+                                                 return_nkeys=True)
         elapsed += time.perf_counter() - t0
-        flop += 4.0 * d * float(nk.sum())
+        flop += per_pair * float(nk.sum())
         done_rows += len(rows)
         nrows = min(nrows * 2, 1024)
-    desc = (f"{done_rows} query rows of head 0 ({'kept tiles in full' if mode == 'block' else 'token-exact keys'}), "
-            f"{int(flop / (4 * d))} computed pairs, {elapsed:.1f} s, including the oracle's brute-force tile "
+    what = "attention" if kind == "fwd" else "dQ (with the S, O, dP it needs)"
+    desc = (f"{what} of {done_rows} query rows of head 0 "
+            f"({'kept tiles in full' if mode == 'block' else 'token-exact keys'}), "
+            f"{int(flop / per_pair)} computed pairs, {elapsed:.1f} s, including the oracle's brute-force tile "
             f"flags of the rows' query tiles")
     return flop / elapsed / 1e12, orc.threads(), desc
 
@@ -225,13 +248,19 @@ def run_reference(args, c, mask):
     per_step = max(1.0, min(8.0, 120.0 / max(n_steps, 1)))
     vals, threads, descs = [], 1, []
     for i in range(n_steps):
-        v, threads, desc = cpu_oracle_sample(args.workload, c["masks"][args.mask], args.mode, c, target_s=per_step)
+        if args.pass_ == "stream":
+            v, threads, desc = cpu_oracle_stream_sample(args.workload, c, c["masks"][args.mask]["window_frames"],
+                                                        target_s=per_step)
+        else:
+            v, threads, desc = cpu_oracle_sample(args.workload, c["masks"][args.mask], args.mode, c,
+                                                 target_s=per_step, kind=args.pass_)
         if i >= args.warmup:
             vals.append(v)
             descs.append(desc)
     value = float(np.median(vals))
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": {"fwd": METRIC, "bwd": METRIC_BWD, "stream": METRIC_STREAM}[args.pass_],
+        "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_desc(args.workload, mask, args.mode, c), "mask": mask["family"],
@@ -239,6 +268,180 @@ def run_reference(args, c, mask):
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": descs[-1] if descs else ""},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def init_ranks():
+    """(world, rank, device): one process per GPU under torchrun (NCCL), else GPU 0."""
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, torch.cuda.current_device()
+
+
+def cpu_oracle_stream_sample(name, c, W, target_s=15.0):
+    """The oracle on sampled query rows of one frame of the sequence under the
+    SWC mask (what one streaming step computes for those rows), head 0."""
+    import oracle
+    orc = oracle.default()
+    s, d = c["s"], c["d"]
+    f = min(c["f"], W + 2)
+    n = f * s
+    spec = oracle.MaskSpec(oracle.SWC, f, s, window_frames=W)
+    seed = synth.config_seed(name)
+    Q, K, V = (synth.normal_bf16(seed, t, (1, 1, n, d)) for t in range(3))
+    rng = np.random.default_rng(seed)
+    rows_all = (f - 1) * s + rng.permutation(s)
+    nrows, done_rows, flop, elapsed = 4, 0, 0.0, 0.0
+    while elapsed < target_s and done_rows < len(rows_all):
+        rows = rows_all[done_rows:done_rows + nrows]
+        t0 = time.perf_counter()
+        _, _, nk = orc.attention_rows(Q, K, V, spec, oracle.TOKEN_EXACT, 1 / math.sqrt(d),
+                                      np.zeros(len(rows), np.int64), rows)
+        elapsed += time.perf_counter() - t0
+        flop += 4.0 * d * float(nk.sum())
+        done_rows += len(rows)
+        nrows = min(nrows * 2, 512)
+    desc = (f"{done_rows} query rows of frame {f - 1} (head 0, SWC W={W}, token-exact over the whole "
+            f"{f}-frame sequence), {int(flop / (4 * d))} computed pairs, {elapsed:.1f} s")
+    return flop / elapsed / 1e12, orc.threads(), desc
+
+
+def run_stream(args, c, mask, world, rank, dev):
+    """One step = one frame through ra_swc_cache_step in steady state (the ring
+    holds W frames): its K, V appended (the oldest evicted) and its s queries
+    attending to the W * s cached tokens."""
+    import torch
+    import torch.distributed as dist
+
+    import static_sparse_attention_b200 as ra
+
+    if mask["family"] != "swc":
+        raise SystemExit("--pass stream needs an SWC mask (e.g. --workload wan_radial --mask 1)")
+    W = mask["window_frames"]
+    B, H, d, s = c["B"], c["H"], c["d"], c["s"]
+    nfr = W + 4  # distinct frames cycled through (inputs larger than L2)
+    seed = synth.config_seed(args.workload)
+    host = [synth.normal_bf16(seed, tid, (B, H, nfr * s, d)) for tid in rank_tensor_ids(rank)]
+    full = [torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).to(f"cuda:{dev}") for h in host]
+    frames = [[t[:, :, i * s:(i + 1) * s].contiguous() for t in full] for i in range(nfr)]
+    del full
+    out = torch.empty((B, H, s, d), dtype=torch.bfloat16, device=f"cuda:{dev}")
+    cache = ra.SwcCache(B, H, d, s, W)
+    stream = torch.cuda.current_stream()
+    scale = 1.0 / math.sqrt(d)
+    counter = [0]
+
+    def step():
+        qf, kf, vf = frames[counter[0] % nfr]
+        counter[0] += 1
+        cache.step(qf, kf, vf, out=out, scale=scale, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(W + args.warmup):  # fill the ring, then warm up in steady state
+        step()
+    torch.cuda.synchronize()
+    assert ra.device_status() == ra.RA_OK
+    flop = 4.0 * d * s * (W * s) * B * H
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(physical_gpu(dev)) as clk:
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    if ra.device_status() != ra.RA_OK:
+        raise SystemExit("device status error after the timed region")
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world, f"cuda:{dev}")
+    ms_per_step = total_ms / args.steps
+    value = flop * args.steps * world / (total_ms / 1e3) / 1e12
+    achieved = flop / (float(np.mean([a.elapsed_time(b) for a, b in zip(starts, ends)])) / 1e3) / 1e12
+    burst, sustained, _, peak_src = measured_peaks()
+    peak = burst if total_ms < 1000.0 else sustained
+
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (torch.from_numpy(h[:, :, :s].copy().view(np.int16)).view(torch.bfloat16).pin_memory()
+                      for h in host)
+        ho = torch.empty((B, H, s, d), dtype=torch.bfloat16).pin_memory()
+        dq, dk, dv = (torch.empty((B, H, s, d), dtype=torch.bfloat16, device=f"cuda:{dev}") for _ in range(3))
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            cache.step(dq, dk, dv, out=out, scale=scale, stream=stream)
+            ho.copy_(out, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 10))
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, f"cuda:{dev}")
+        e2e = {"value": flop * e2e_steps * world / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms / e2e_steps, "h2d_bytes_per_step": 3 * out.numel() * 2,
+               "d2h_bytes_per_step": out.numel() * 2,
+               "path": "pinned host frame Q,K,V -> device, ra_swc_cache_step, device -> pinned host O"}
+    cache.free()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        val, threads, desc = cpu_oracle_stream_sample(args.workload, c, W)
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+    ring_bytes = 2 * B * H * W * s * d * 2
+    line = {
+        "metric": METRIC_STREAM, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": f"{args.workload} frames streamed through the SWC key/value ring cache: s={s}, W={W}, "
+                        f"B={B}, H={H}, d={d}, bf16 Q,K,V iid N(0,1), steady state (ring full)",
+            "pass": "stream", "frame_tokens": s, "window_frames": W, "cached_tokens": W * s,
+            "l2": f"inputs larger than L2: ring K+V = {ring_bytes / 1e9:.2f} GB per GPU vs 126 MB L2",
+            "flop_definition": "4*d per (query, cached key) pair per head: s * W * s pairs per head per frame",
+            "parallelism": f"{world} independent streams (one per GPU), no collective",
+        },
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 {'burst' if total_ms < 1000.0 else 'sustained'}",
+                     "kernel": "attn_fwd_kernel<%d> over the ring (plus two 2D copies of the frame's K, V)" % d,
+                     "flop_per_launch": flop},
+        "clocks": clk.summary(),
+        "gpu_launches": args.steps,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
 
@@ -258,17 +461,10 @@ def main():
 
     import static_sparse_attention_b200 as ra
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
-    else:
-        torch.cuda.set_device(0)
-    dev = torch.cuda.current_device()
+    world, rank, dev = init_ranks()
+    if args.pass_ == "stream":
+        run_stream(args, c, mask, world, rank, dev)
+        return
 
     B, H, d = c["B"], c["H"], c["d"]
     n = c["f"] * c["s"]
@@ -280,13 +476,30 @@ def main():
     o = torch.empty_like(q)
     m = ra.build_mask(mask, c["f"], c["s"], c["grid"])
     info = m.info
-    flop = flops_per_call(info, c, args.mode)
+    bwd = args.pass_ == "bwd"
+    flop = flops_per_call(info, c, args.mode, args.pass_)
     scale = 1.0 / math.sqrt(d)
     stream = torch.cuda.current_stream()
     bytes_qkvo = 4 * q.numel() * 2
+    launches_per_step = 1
 
-    def step():
-        ra.attention_fwd(q, k, v, m, scale=scale, mode=args.mode, out=o, stream=stream)
+    if bwd:
+        # the backward's inputs: this rank's seeded dO, and O and lse from the forward
+        host.append(synth.normal_bf16(seed, synth.DOUT_TENSOR_ID + rank, shape))
+        do = torch.from_numpy(host[3].view(np.int16)).view(torch.bfloat16).to(f"cuda:{dev}")
+        lse = torch.empty((B, H, n), dtype=torch.float32, device=f"cuda:{dev}")
+        ra.attention_fwd(q, k, v, m, scale=scale, mode=args.mode, out=o, lse=lse, stream=stream)
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+        ws = torch.empty((B, H, n), dtype=torch.float32, device=f"cuda:{dev}")
+        bytes_qkvo = 8 * q.numel() * 2 + 2 * lse.numel() * 4  # Q K V O dO in, dQ dK dV out, lse in, D
+        launches_per_step = 3  # D = rowsum(dO * O), dQ pass, dK / dV pass
+
+        def step():
+            ra.attention_bwd(q, k, v, o, do, lse, m, scale=scale, mode=args.mode, dq=dq, dk=dk, dv=dv,
+                             workspace=ws, stream=stream)
+    else:
+        def step():
+            ra.attention_fwd(q, k, v, m, scale=scale, mode=args.mode, out=o, stream=stream)
 
     def barrier():
         if world > 1:
@@ -327,16 +540,53 @@ def main():
     timed_alone = total_ms < 1000.0
     peak = burst if timed_alone else sustained
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": recorded_traffic(args.workload, args.mode, mask["family"]),
+                "frac": achieved / peak,
+                "traffic": recorded_traffic(args.workload, args.mode, mask["family"], args.pass_),
                 "peak_source": f"{peak_src} bf16 {'burst' if timed_alone else 'sustained'} (MEASURED_PEAKS.json)"
                 if peak_src == "measured" else "fallback 1.59 PFLOP/s burst / 1.4 sustained",
-                "kernel": "attn_fwd_kernel<%d>" % d,
+                "kernel": ("attn_fwd_kernel<%d>" % d) if not bwd else
+                ("ra_attention_bwd call: bwd_dot_kernel<%d> + bwd_kernel<%d, dQ> + bwd_kernel<%d, dK dV>" % (d, d, d)),
                 "flop_per_launch": flop,
                 "algorithmic_bytes_per_launch": bytes_qkvo}
 
     # ---- end to end: host buffers through the C ABI (H2D + kernel + D2H per step)
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and bwd:
+        # pinned host Q, K, V, O, dO, lse -> device, the backward, dQ, dK, dV -> pinned host
+        hosts = [torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).pin_memory() for h in host]
+        hosts.append(torch.from_numpy(host[0].view(np.int16)).view(torch.bfloat16).pin_memory())  # O slot
+        hosts[4].copy_(o.cpu())
+        hl = lse.cpu().pin_memory()
+        houts = [torch.empty(shape, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+        devs = [q, k, v, do, o]
+
+        def e2e_step():
+            for hsrc, dst in zip(hosts, devs):
+                dst.copy_(hsrc, non_blocking=True)
+            lse.copy_(hl, non_blocking=True)
+            step()
+            for hdst, src in zip(houts, (dq, dk, dv)):
+                hdst.copy_(src, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 10))
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, f"cuda:{dev}")
+        e2e = {"value": flop * e2e_steps * world / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms / e2e_steps, "h2d_bytes_per_step": 5 * q.numel() * 2 + lse.numel() * 4,
+               "d2h_bytes_per_step": 3 * q.numel() * 2,
+               "path": "pinned host Q,K,V,O,dO,lse -> device, ra_attention_bwd, device -> pinned host dQ,dK,dV"}
+        del hosts, houts, hl
+    if not args.no_e2e and not bwd:
         hq, hk, hv = (torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).pin_memory() for h in host)
         ho = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
         e2e_steps = max(3, min(args.steps, 10))
@@ -360,7 +610,7 @@ def main():
 
     # ---- the same kernel with the dense mask on the same inputs (reference point)
     dense_ref = None
-    if not args.no_dense_ref and mask["family"] != "dense":
+    if not args.no_dense_ref and mask["family"] != "dense" and not bwd:
         md = ra.build_mask(dict(family="dense"), c["f"], c["s"])
         dflop = flops_per_call(md.info, c, "block")
         for _ in range(2):
@@ -384,27 +634,31 @@ def main():
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        val, threads, desc = cpu_oracle_sample(args.workload, mask, args.mode, c)
+        val, threads, desc = cpu_oracle_sample(args.workload, mask, args.mode, c, kind=args.pass_)
         cpu = {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
 
     tile_total = info["nb"] ** 2
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {
             "workload": workload_desc(args.workload, mask, args.mode, c),
-            "mask": mask["family"], "mode": args.mode, "global_batch": B * world, "heads": H, "seq_len": n,
+            "mask": mask["family"], "mode": args.mode, "pass": args.pass_, "global_batch": B * world, "heads": H,
+            "seq_len": n,
             "head_dim": d, "parallelism": f"{world} independent problems (one per GPU), no collective",
-            "l2": f"inputs larger than L2: Q+K+V+O = {bytes_qkvo / 1e9:.2f} GB per GPU vs 126 MB L2",
+            "l2": f"inputs larger than L2: {'Q+K+V+O' if not bwd else 'Q+K+V+O+dO+dQ+dK+dV'} = "
+                  f"{bytes_qkvo / 1e9:.2f} GB per GPU vs 126 MB L2",
             "kept_tiles": info["nnz"], "tile_sparsity": 1.0 - info["nnz"] / tile_total,
             "token_sparsity": 1.0 - info["kept_pairs"] / float(n) ** 2,
-            "flop_definition": "4*d per computed pair per head; block mode computes every valid pair of kept tiles",
+            "flop_definition": ("4*d" if not bwd else "10*d (S, dP, dQ, dK, dV)") +
+                               " per computed pair per head; block mode computes every valid pair of kept tiles",
         },
         "pct_of_peak": 100.0 * roofline["frac"],
         "roofline": roofline,
         "clocks": clk.summary(),
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * launches_per_step,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "dense_same_kernel": dense_ref,

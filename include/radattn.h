@@ -107,7 +107,9 @@ typedef struct {
  * Arrays (device, owned by the mask): row_ptr int32[nb + 1]; col_idx int32[nnz]
  * (ascending within a row); count int32[nnz] (kept pairs of the tile);
  * flag uint8[nnz] (RA_TILE_FULL iff count == 128 * 128).  A tile is kept iff it
- * holds at least one kept valid pair.
+ * holds at least one kept valid pair.  The mask also holds the transposed
+ * block-CSR (for each key tile its query tiles: col_ptr, row_idx, tflag), which
+ * ra_attention_bwd walks for dK and dV.
  * Synchronises `stream` once (to size the arrays).  Limits: f, s >= 1,
  * n <= 2^31 - 1 and nb * nb <= 2^31 - 1.  INVALID_ARG on bad parameters,
  * OUT_OF_MEMORY / CUDA on device failures (nothing is leaked).
@@ -155,6 +157,12 @@ ra_status ra_mask_copy_to_host(const ra_mask* m, int* row_ptr, int* col_idx, int
 ra_status ra_mask_device_arrays(const ra_mask* m, const int** row_ptr, const int** col_idx, const int** count,
                                 const unsigned char** flag);
 
+/* Copy the transposed block-CSR (per key tile, the query tiles that keep it, in
+ * ascending order, with the tile's FULL / PARTIAL flag) to caller-allocated host
+ * arrays: col_ptr int32[nb + 1], row_idx int32[nnz], tflag uint8[nnz].  The
+ * backward pass walks it.  Any pointer may be NULL.  Synchronous. */
+ra_status ra_mask_copy_transpose_to_host(const ra_mask* m, int* col_ptr, int* row_idx, unsigned char* tflag);
+
 /* Release a mask (NULL is ignored).  Synchronises the device first. */
 void ra_mask_free(ra_mask* m);
 
@@ -186,6 +194,61 @@ ra_status ra_attention_fwd(const void* Q, const void* K, const void* V, void* O,
 ra_status ra_attention_fwd_host(const void* Q_host, const void* K_host, const void* V_host, void* O_host,
                                 void* Q_dev, void* K_dev, void* V_dev, void* O_dev, int B, int H, int d,
                                 const ra_mask* m, float scale, int mode, ra_stream stream);
+
+/*
+ * ra_attention_bwd -- gradients of ra_attention_fwd ("Radial Attention ..."
+ * eq. 2 with the 128 x 128 tile mask of sec. 6).  The page trains its LoRA
+ * adapters through the sparse attention (sec. 6: block-sparse FlashAttention-2
+ * for training; sec. 7: training speedups) without writing the backward out;
+ * these are the standard softmax-attention gradients restricted to the kept pairs.  With
+ * P = exp(scale * Q K^T + M - lse), D_i = <dO_i, O_i>, dS = P * (dO V^T - D):
+ *   dQ = scale * dS K,   dK = scale * dS^T Q,   dV = P^T dO.
+ *   Q, K, V, O, dO : device, bf16 [B, H, n, d], contiguous, 16-byte aligned;
+ *                    O is the forward's output for the same Q, K, V, m, mode.
+ *   lse            : device fp32 [B, H, n], the forward's log-sum-exp.
+ *   dQ, dK, dV     : device, bf16 [B, H, n, d], written (no aliasing with the inputs).
+ *   D_workspace    : device fp32 [B, H, n], caller-owned scratch (receives D).
+ *   d, m, scale, mode : as for ra_attention_fwd (same values as the forward).
+ * dQ walks the block-CSR rows, dK and dV the transposed block-CSR; no atomics,
+ * so the result is deterministic.  Asynchronous on `stream`; no allocation.
+ */
+ra_status ra_attention_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                           const float* lse, void* dQ, void* dK, void* dV, float* D_workspace, int B, int H, int d,
+                           const ra_mask* m, float scale, int mode, ra_stream stream);
+
+/*
+ * Streaming sliding-window causal attention with a key/value ring cache
+ * (the Vera 1.1 temporal module, sec. 3.1: during inference the K and V of the
+ * frames inside the window are cached; as the window moves on, the oldest
+ * frame's K and V are evicted and the new frame's added, so memory stays fixed).
+ *
+ * ra_swc_cache_create -- a cache for B x H heads of d (64 or 128) channels,
+ *   s tokens per frame and a window of W = window_frames frames.  Allocates two
+ *   device rings of B * H * W * s * d bf16 (K and V) plus a few KB of tile lists;
+ *   synchronous.  The cache is bound to the current device.
+ * ra_swc_cache_step -- feed the next frame (index i = frames fed so far):
+ *   Q_frame, K_frame, V_frame : device bf16 [B, H, s, d], contiguous, 16-byte aligned.
+ *   O_frame                   : device bf16 [B, H, s, d], written.
+ *   lse                       : NULL or device fp32 [B, H, s] (natural log).
+ *   The frame's K and V replace frame i - W's in the ring; then O_frame is the
+ *   attention of the frame's queries over every token of frames max(0, i-W+1) .. i,
+ *   the rows of frame i of the SWC mask (RA_MASK_SWC, same W) over the whole
+ *   sequence.  Asynchronous on `stream`; steps must be ordered (one stream).
+ * ra_swc_cache_info  -- frames fed so far and frames held (min(fed, W)).  Host only.
+ * ra_swc_cache_copy_rings_to_host -- copy the K and V rings, each
+ *   [B, H, W * s, d] bf16 with frame i in slot i mod W, to host arrays (either
+ *   may be NULL).  Synchronises the device.
+ * ra_swc_cache_reset -- forget every frame (the next step is frame 0).  Host only.
+ * ra_swc_cache_free  -- synchronise the device and release the cache (NULL ignored).
+ */
+typedef struct ra_swc_cache ra_swc_cache;
+ra_status ra_swc_cache_create(int B, int H, int d, int s, int window_frames, ra_swc_cache** out);
+ra_status ra_swc_cache_step(ra_swc_cache* c, const void* Q_frame, const void* K_frame, const void* V_frame,
+                            void* O_frame, float scale, float* lse, ra_stream stream);
+ra_status ra_swc_cache_info(const ra_swc_cache* c, long long* frames_seen, int* frames_held);
+ra_status ra_swc_cache_copy_rings_to_host(const ra_swc_cache* c, void* K_host, void* V_host);
+ra_status ra_swc_cache_reset(ra_swc_cache* c);
+void ra_swc_cache_free(ra_swc_cache* c);
 
 /* Synchronise `stream`, then read and clear the current device's error word.
  * RA_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since the last call. */

@@ -113,7 +113,7 @@ def load_library(path: str):
                                          vp]
     lib.oracle_attention_bwd.restype = None
     lib.oracle_attention_bwd_query_rows.argtypes = [vp, vp, vp, vp, c_int, i64, c_int, P, c_int, ctypes.c_double,
-                                                    i64, vp, vp, vp, vp, vp]
+                                                    i64, vp, vp, vp, vp, vp, vp]
     lib.oracle_attention_bwd_query_rows.restype = None
     lib.oracle_attention_bwd_key_rows.argtypes = [vp, vp, vp, vp, c_int, i64, c_int, P, c_int, ctypes.c_double,
                                                   vp, i64, vp, vp, vp]
@@ -227,8 +227,10 @@ class Oracle:
         return tuple(out)
 
 
-    def attention_bwd_query_rows(self, Q, K, V, dO, spec: MaskSpec, mode: int, scale: float, row_bh, row_q):
-        """fp64 dQ of the listed query rows (b*H + h, q); [rows, d].  O(keys * d) per row."""
+    def attention_bwd_query_rows(self, Q, K, V, dO, spec: MaskSpec, mode: int, scale: float, row_bh, row_q,
+                                 return_nkeys: bool = False):
+        """fp64 dQ of the listed query rows (b*H + h, q); [rows, d].  O(keys * d) per row.
+        With return_nkeys, also each row's key count."""
         Q, K, V, dO = (np.ascontiguousarray(t) for t in (Q, K, V, dO))
         assert Q.dtype == K.dtype == V.dtype == dO.dtype and Q.dtype in _IN_DTYPES
         n, d = Q.shape[-2], Q.shape[-1]
@@ -244,12 +246,14 @@ class Oracle:
             tile_flags = np.zeros(1, dtype=np.uint8)
             slot = np.zeros(max(nrows, 1), dtype=np.int32)
         dQ = np.empty((nrows, d), dtype=np.float64)
+        nkeys = np.empty(max(nrows, 1), dtype=np.int64)
         sp = spec.c()
         self.lib.oracle_attention_bwd_query_rows(Q.ctypes.data, K.ctypes.data, V.ctypes.data, dO.ctypes.data,
                                                  _IN_DTYPES[Q.dtype], n, d, ctypes.byref(sp), mode, float(scale),
                                                  nrows, row_bh.ctypes.data, row_q.ctypes.data,
-                                                 tile_flags.ctypes.data, slot.ctypes.data, dQ.ctypes.data)
-        return dQ
+                                                 tile_flags.ctypes.data, slot.ctypes.data, dQ.ctypes.data,
+                                                 nkeys.ctypes.data)
+        return (dQ, nkeys[:nrows]) if return_nkeys else dQ
 
     def attention_bwd_key_rows(self, Q, K, V, dO, spec: MaskSpec, mode: int, scale: float, keys):
         """fp64 dK, dV of the listed key rows of ONE (b, h) slice: Q, K, V, dO are

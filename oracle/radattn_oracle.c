@@ -421,12 +421,13 @@ static long long or_row_scores(const void* Q, const void* K, int dtype, long lon
  * (dQ_i = scale sum_j P_ij (<dO_i, V_j> - D_i) K_j, D_i = <dO_i, O_i>), one row
  * at a time in O(keys * d): for sampled rows of workloads too large for the
  * whole backward.  Rows and tile flags as in oracle_attention_rows; dQ is
- * [nrows, d] fp64.
+ * [nrows, d] fp64; nkeys (may be NULL) receives each row's key count.
  */
 void oracle_attention_bwd_query_rows(const void* Q, const void* K, const void* V, const void* dO, int dtype,
                                      long long n, int d, const or_spec* sp, int mode, double scale, long long nrows,
                                      const long long* row_bh, const long long* row_q,
-                                     const unsigned char* tile_flags, const int* row_tile_slot, double* dQ)
+                                     const unsigned char* tile_flags, const int* row_tile_slot, double* dQ,
+                                     long long* nkeys)
 {
     long long nb = (n + OR_TILE - 1) / OR_TILE;
 #pragma omp parallel
@@ -442,6 +443,8 @@ void oracle_attention_bwd_query_rows(const void* Q, const void* K, const void* V
             const unsigned char* flags = mode == OR_TOKEN_EXACT ? NULL : tile_flags + (long long)row_tile_slot[r] * nb;
             double lse;
             long long m = or_row_scores(Q, K, dtype, n, d, sp, mode, scale, q, flags, qoff, kvbase, idx, x, &lse);
+            if (nkeys)
+                nkeys[r] = m;
             for (int c = 0; c < d; c++)
                 dQ[r * d + c] = 0.0;
             if (m == 0)

@@ -58,8 +58,16 @@ _SIGS = {
     "ra_mask_device_arrays": ([_MaskP, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
                                ctypes.POINTER(_vp)], _i),
     "ra_mask_free": ([_MaskP], None),
+    "ra_mask_copy_transpose_to_host": ([_MaskP, _vp, _vp, _vp], _i),
     "ra_attention_fwd": ([_vp, _vp, _vp, _vp, _i, _i, _i, _MaskP, _f, _i, _vp, _vp], _i),
     "ra_attention_fwd_host": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _MaskP, _f, _i, _vp], _i),
+    "ra_attention_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _MaskP, _f, _i, _vp], _i),
+    "ra_swc_cache_create": ([_i, _i, _i, _i, _i, ctypes.POINTER(_vp)], _i),
+    "ra_swc_cache_step": ([_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp], _i),
+    "ra_swc_cache_info": ([_vp, ctypes.POINTER(_ll), ctypes.POINTER(_i)], _i),
+    "ra_swc_cache_copy_rings_to_host": ([_vp, _vp, _vp], _i),
+    "ra_swc_cache_reset": ([_vp], _i),
+    "ra_swc_cache_free": ([_vp], None),
     "ra_get_device_status": ([_vp], _i),
     "ra_get_device_error_site": ([ctypes.POINTER(_i), ctypes.POINTER(_i)], _i),
     "ra_selftest_wait_timeout": ([_ll, _vp], _i),
@@ -132,6 +140,17 @@ class Mask:
                                    flag.ctypes.data), "ra_mask_copy_to_host")
         return dict(row_ptr=row_ptr, col_idx=col_idx, count=count, flag=flag, nnz=nnz)
 
+    def transpose_to_host(self) -> dict:
+        """The transposed block-CSR: col_ptr, row_idx, tflag."""
+        import numpy as np
+        nb, nnz = self.info["nb"], self.info["nnz"]
+        col_ptr = np.empty(nb + 1, dtype=np.int32)
+        row_idx = np.empty(nnz, dtype=np.int32)
+        tflag = np.empty(nnz, dtype=np.uint8)
+        check(ra_mask_copy_transpose_to_host(self.handle, col_ptr.ctypes.data, row_idx.ctypes.data,
+                                             tflag.ctypes.data), "ra_mask_copy_transpose_to_host")
+        return dict(col_ptr=col_ptr, row_idx=row_idx, tflag=tflag)
+
     def free(self) -> None:
         if getattr(self, "_h", None) is not None:
             ra_mask_free(self._h)
@@ -188,6 +207,101 @@ def attention_fwd_host(q_host, k_host, v_host, o_host, q_dev, k_dev, v_dev, o_de
                                 q_dev.data_ptr(), k_dev.data_ptr(), v_dev.data_ptr(), o_dev.data_ptr(), B, H, d,
                                 mask.handle, scale, mode, _stream_handle(stream)), "ra_attention_fwd_host")
     return o_host
+
+
+def attention_bwd(q, k, v, out, dout, lse, mask: Mask, scale: float | None = None, mode="block",
+                  dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of attention_fwd given its output `out`, its fp32 `lse` and the
+    output gradient `dout` (all bf16 [B, H, n, d] except lse [B, H, n])."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        _check_bf16_cuda(name, t)
+    B, H, n, d = q.shape
+    if any(t.shape != q.shape for t in (k, v, out, dout)) or n != mask.n:
+        raise ValueError("q, k, v, out, dout must share shape [B, H, n, d] with n equal to the mask's n")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, n) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 tensor [B, H, n]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_bf16_cuda(name, t)
+        if t.shape != q.shape:
+            raise ValueError(f"{name} must have shape [B, H, n, d]")
+    if workspace is None:
+        workspace = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
+    if workspace.dtype != torch.float32 or workspace.numel() < B * H * n or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous fp32 tensor of at least B * H * n elements")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    mode = MODES[mode] if isinstance(mode, str) else int(mode)
+    check(ra_attention_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                           lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                           B, H, d, mask.handle, scale, mode, _stream_handle(stream)), "ra_attention_bwd")
+    return dq, dk, dv
+
+
+class SwcCache:
+    """Streaming sliding-window causal attention with a key/value ring cache of
+    `window_frames` frames of `s` tokens for B x H heads of d channels."""
+
+    def __init__(self, B: int, H: int, d: int, s: int, window_frames: int):
+        h = ctypes.c_void_p()
+        check(ra_swc_cache_create(B, H, d, s, window_frames, ctypes.byref(h)), "ra_swc_cache_create")
+        self._h = h
+        self.B, self.H, self.d, self.s, self.W = B, H, d, s, window_frames
+
+    @property
+    def handle(self):
+        if self._h is None:
+            raise ValueError("cache was freed")
+        return self._h
+
+    def step(self, q, k, v, out=None, lse=None, scale: float | None = None, stream=None):
+        """Feed the next frame (q, k, v bf16 [B, H, s, d]); returns its output."""
+        import torch
+        for name, t in (("q", q), ("k", k), ("v", v)):
+            _check_bf16_cuda(name, t)
+            if tuple(t.shape) != (self.B, self.H, self.s, self.d):
+                raise ValueError(f"{name} must have shape [B, H, s, d]")
+        if out is None:
+            out = torch.empty_like(q)
+        _check_bf16_cuda("out", out)
+        if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (self.B, self.H, self.s)
+                                or not lse.is_contiguous()):
+            raise ValueError("lse must be a contiguous fp32 tensor [B, H, s]")
+        scale = 1.0 / math.sqrt(self.d) if scale is None else float(scale)
+        check(ra_swc_cache_step(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), scale,
+                                None if lse is None else lse.data_ptr(), _stream_handle(stream)), "ra_swc_cache_step")
+        return out
+
+    @property
+    def info(self) -> dict:
+        seen, held = ctypes.c_longlong(), ctypes.c_int()
+        check(ra_swc_cache_info(self.handle, ctypes.byref(seen), ctypes.byref(held)), "ra_swc_cache_info")
+        return dict(frames_seen=seen.value, frames_held=held.value)
+
+    def rings_to_host(self):
+        """(K ring, V ring) as uint16 bf16 bit patterns [B, H, W * s, d]; frame i in slot i mod W."""
+        import numpy as np
+        shape = (self.B, self.H, self.W * self.s, self.d)
+        k, v = np.empty(shape, dtype=np.uint16), np.empty(shape, dtype=np.uint16)
+        check(ra_swc_cache_copy_rings_to_host(self.handle, k.ctypes.data, v.ctypes.data),
+              "ra_swc_cache_copy_rings_to_host")
+        return k, v
+
+    def reset(self) -> None:
+        check(ra_swc_cache_reset(self.handle), "ra_swc_cache_reset")
+
+    def free(self) -> None:
+        if getattr(self, "_h", None) is not None:
+            ra_swc_cache_free(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
 
 
 def device_status(stream=None) -> int:

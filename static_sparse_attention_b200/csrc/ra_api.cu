@@ -1,9 +1,12 @@
-// ra_api.cu -- status strings, per-thread error details and library settings.
+// ra_api.cu -- status strings, per-thread error details, library settings and
+// TMA tensor maps.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 
 #include "ra_internal.h"
 
@@ -32,6 +35,53 @@ ra_status cuda_fail(cudaError_t e, const char* what)
 }
 
 unsigned long long wait_timeout_ns() { return g_timeout_ns.load(std::memory_order_relaxed); }
+
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+}  // namespace
+
+// [B*H, head_rows, d] bf16 as a 3D tensor (d, rows, B*H): boxes of box_rows
+// rows x 64 columns, 128-byte swizzle; rows beyond `rows` read as zero.
+ra_status make_map_rows(CUtensorMap* map, const void* base, int BH, int rows, int head_rows, int d, int box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return fail(RA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    if (rows < 1 || rows > head_rows)
+        return fail(RA_ERR_INVALID_ARG, "tensor map rows %d outside [1, %d]", rows, head_rows);
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(head_rows) * d * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(RA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return RA_OK;
+}
+
+ra_status make_map(CUtensorMap* map, const void* base, int BH, int n, int d, int box_rows)
+{
+    return make_map_rows(map, base, BH, n, n, d, box_rows);
+}
 
 }  // namespace ra
 

@@ -103,8 +103,9 @@ enum : int {
 };
 
 struct FwdParams {
-    MaskGeom g;
-    int nb, H, mode;
+    MaskGeom g;        // query rows: g.n; the family mask of token-exact partial tiles
+    int nb, H, mode;   // nb: query tiles (the grid)
+    int nk, nbk;       // key rows and key tiles (n and nb for self-attention)
     const int* row_ptr;
     const int* col_idx;
     const unsigned char* flag;
@@ -113,19 +114,6 @@ struct FwdParams {
     float scale_log2;  // scale * log2(e)
     unsigned long long timeout_ns;
 };
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
-{
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
-__device__ __forceinline__ float fast_exp2(float x)
-{
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 // ---- packed fp32 pairs (sm_100 f32x2 instructions) -------------------------
 __device__ __forceinline__ uint64_t f2pack(float lo, float hi)
@@ -236,18 +224,6 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&r)[32], float c, floa
 #define RA_EMU_PER_32 0
 #endif
 constexpr int EMU_PER_32 = RA_EMU_PER_32;
-
-// Wait without the CTA abort flag: used only to drain in-flight copies and
-// MMAs before the CTA releases its memory.
-__device__ bool drain_wait(uint32_t bar, uint32_t parity, unsigned long long timeout_ns)
-{
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > timeout_ns)
-            return false;
-    }
-    return true;
-}
 
 // SPLIT_P: P is kept as hi + lo bf16 pairs (P = hi + lo to ~16 bits) and
 // P V runs as two MMAs; used for masks whose rows hold few keys, where the
@@ -392,7 +368,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
         const bool row_valid = row < n;
         const int qi = row_valid ? row / p.g.s : 0, qk = row_valid ? row % p.g.s : 0;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        const bool tail = (n % TILE) != 0;
+        const bool tail = (p.nk % TILE) != 0;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
@@ -405,19 +381,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
             const uint32_t s_col = s_col_of(buf);
             if (half == 0) {
                 // Mask of the whole tile: token-exact partial tiles use the
-                // family's element mask; the tail key tile masks keys >= n.
+                // family's element mask; the tail key tile masks keys >= nk.
                 const int kb = next_kb;
                 const bool use_family = p.mode == RA_MODE_TOKEN_EXACT && next_flag != RA_TILE_FULL;
                 if (i + 1 < L_row) {
                     next_kb = p.col_idx[row_start + i + 1];
                     next_flag = p.flag[row_start + i + 1];
                 }
-                masked = use_family || (tail && kb == p.nb - 1);
+                masked = use_family || (tail && kb == p.nbk - 1);
                 if (masked) {
                     if (use_family && row_valid) {
                         row_keep_mask(p.g, qi, qk, kb * TILE, mk[0], mk[1], mk[2], mk[3]);
                     } else {
-                        const int valid_cols = min(TILE, n - kb * TILE);
+                        const int valid_cols = min(TILE, p.nk - kb * TILE);
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
                             const int v = valid_cols - 32 * c;
@@ -604,44 +580,6 @@ __global__ void wait_selftest_kernel(unsigned long long timeout_ns)
     }
 }
 
-// ------------------------------------------------------------ tensor maps
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    });
-    return fn;
-}
-
-// [B*H, n, d] bf16, boxes of 128 rows x 64 columns, 128-byte swizzle; rows
-// beyond n read as zero.
-ra_status make_map(CUtensorMap* map, const void* base, int BH, int n, int d, int box_rows)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn)
-        return fail(RA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(BH)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(n) * d * 2};
-    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS)
-        return fail(RA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-    return RA_OK;
-}
-
 template <int D, bool SPLIT_P>
 ra_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p, int B,
                      cudaStream_t cs)
@@ -666,7 +604,6 @@ ra_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 constexpr long long SPLIT_P_MAX_KEYS_PER_ROW = 4096;
 std::atomic<int> g_pv_policy{RA_PV_AUTO};
 
-bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
 ra_status check_fwd_args(const void* Q, const void* K, const void* V, const void* O, int B, int H, int d,
                          const ra_mask* m, float scale, int mode)
@@ -719,6 +656,8 @@ extern "C" ra_status ra_attention_fwd(const void* Q, const void* K, const void* 
     std::memset(&p, 0, sizeof p);
     p.g = m->geom;
     p.nb = m->nb;
+    p.nk = n;
+    p.nbk = m->nb;
     p.H = H;
     p.mode = mode;
     p.row_ptr = m->row_ptr;
@@ -737,6 +676,44 @@ extern "C" ra_status ra_attention_fwd(const void* Q, const void* K, const void* 
         return split ? launch_fwd<64, true>(mq, mk, mv, p, B, cs) : launch_fwd<64, false>(mq, mk, mv, p, B, cs);
     return split ? launch_fwd<128, true>(mq, mk, mv, p, B, cs) : launch_fwd<128, false>(mq, mk, mv, p, B, cs);
 }
+
+namespace ra {
+ra_status attention_fwd_rect(const void* Q, const void* K, const void* V, void* O, int B, int H, int d, int nq,
+                             int nk, int k_head_rows, const int* row_ptr, const int* col_idx,
+                             const unsigned char* flag, int nbq, float scale, float* lse, cudaStream_t cs)
+{
+    ra_status st;
+    CUtensorMap mq, mk, mv;
+    const int BH = B * H;
+    if ((st = make_map(&mq, Q, BH, nq, d, TILE)) != RA_OK ||
+        (st = make_map_rows(&mk, K, BH, nk, k_head_rows, d, HALF)) != RA_OK ||
+        (st = make_map_rows(&mv, V, BH, nk, k_head_rows, d, HALF)) != RA_OK)
+        return st;
+    FwdParams p;
+    std::memset(&p, 0, sizeof p);
+    p.g.family = FAM_DENSE;
+    p.g.f = 1;
+    p.g.s = nq;
+    p.g.n = nq;
+    p.nb = nbq;
+    p.nk = nk;
+    p.nbk = (nk + TILE - 1) / TILE;
+    p.H = H;
+    p.mode = RA_MODE_BLOCK;
+    p.row_ptr = row_ptr;
+    p.col_idx = col_idx;
+    p.flag = flag;
+    p.O = static_cast<__nv_bfloat16*>(O);
+    p.lse = lse;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.timeout_ns = wait_timeout_ns();
+    const int policy = g_pv_policy.load(std::memory_order_relaxed);
+    const bool split = policy == RA_PV_SPLIT || (policy == RA_PV_AUTO && nk < SPLIT_P_MAX_KEYS_PER_ROW);
+    if (d == 64)
+        return split ? launch_fwd<64, true>(mq, mk, mv, p, B, cs) : launch_fwd<64, false>(mq, mk, mv, p, B, cs);
+    return split ? launch_fwd<128, true>(mq, mk, mv, p, B, cs) : launch_fwd<128, false>(mq, mk, mv, p, B, cs);
+}
+}  // namespace ra
 
 extern "C" ra_status ra_attention_fwd_host(const void* Q_host, const void* K_host, const void* V_host, void* O_host,
                                            void* Q_dev, void* K_dev, void* V_dev, void* O_dev, int B, int H, int d,
@@ -757,6 +734,18 @@ extern "C" ra_status ra_attention_fwd_host(const void* Q_host, const void* K_hos
     RA_CUDA_TRY(cudaMemcpyAsync(O_host, O_dev, bytes, cudaMemcpyDeviceToHost, cs));
     return RA_OK;
 }
+
+namespace ra {
+ra_status device_error_word(int** out)
+{
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_err);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+    *out = static_cast<int*>(p);
+    return RA_OK;
+}
+}  // namespace ra
 
 extern "C" ra_status ra_get_device_status(ra_stream stream)
 {

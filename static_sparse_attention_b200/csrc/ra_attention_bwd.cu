@@ -1,0 +1,485 @@
+// ra_attention_bwd.cu -- backward of the block-sparse attention for sm_100a.
+//
+// Gradients of O = softmax(scale * Q K^T + M) V ("Radial Attention ..." eq. 2)
+// over the kept 128 x 128 tiles (sec. 6), given dO and the forward's
+// log-sum-exp L:
+//   P = exp(scale * S - L),  D_i = <dO_i, O_i>,  dP = dO V^T,  dS = P (dP - D)
+//   dQ = scale dS K,   dK = scale dS^T Q,   dV = P^T dO.
+// Deterministic: no atomics, each output tile is owned by one CTA.
+//
+//   bwd_dot_kernel   D = rowsum(dO * O) (fp32), one warp per row.
+//   bwd_kernel<D, false>  one CTA per query tile, walking its block-CSR row:
+//       S = Q K^T and dP = dO V^T (tcgen05.mma into TMEM), dS (registers,
+//       bf16 back into TMEM), dQ += dS K (A = dS from TMEM).
+//   bwd_kernel<D, true>   one CTA per key tile, walking the transposed CSR:
+//       S^T = K Q^T and dP^T = V dO^T, P^T and dS^T (bf16 into TMEM),
+//       dV += P^T dO and dK += dS^T Q.
+// Both recompute P from L instead of storing it.  192 threads: warps 0-3 own
+// one tile row each per thread (TMEM lane = row), warp 4 issues the TMA loads
+// (two resident tiles, two 2-stage rings), warp 5 allocates TMEM and issues
+// the MMAs.  TMEM columns: S at 0, dP at 128, the accumulators at 256 and 384.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "ra_internal.h"
+#include "ra_sm100.cuh"
+
+namespace ra {
+namespace {
+
+constexpr int BWD_THREADS = 192;
+constexpr uint32_t BWD_TMEM_COLS = 512;
+constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC0 = 256, COL_ACC1 = 384;
+constexpr float LOG2E = 1.4426950408889634f;
+
+enum : int { BSITE_RES = 21, BSITE_X_EMPTY, BSITE_Y_EMPTY, BSITE_X_FULL, BSITE_Y_FULL, BSITE_S_FULL, BSITE_P_FULL,
+             BSITE_ACC, BSITE_FINAL };
+
+template <int D>
+struct BLayout {
+    static constexpr int CHUNKS = D / 64;
+    static constexpr int CHUNK_BYTES = TILE * 128;
+    static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;
+    static constexpr int STAGES = 2;
+    static constexpr int R0_OFF = 0;                              // resident: Q (dQ pass) or K (dK/dV pass)
+    static constexpr int R1_OFF = R0_OFF + TILE_BYTES;            // resident: dO or V
+    static constexpr int X_OFF = R1_OFF + TILE_BYTES;             // ring: K_j or Q_i
+    static constexpr int Y_OFF = X_OFF + STAGES * TILE_BYTES;     // ring: V_j or dO_i
+    static constexpr int BAR_OFF = Y_OFF + STAGES * TILE_BYTES;
+    static constexpr int STAT_OFF = BAR_OFF + 256;                // [2 buffers][L2, D][128] floats
+    static constexpr int SMEM_NEEDED = STAT_OFF + 2 * 2 * TILE * 4 + 1024;
+    static constexpr int SMEM_BYTES = SMEM_NEEDED > 120 * 1024 ? SMEM_NEEDED : 120 * 1024;
+};
+
+enum : int {
+    BB_RES_FULL = 0,
+    BB_X_FULL = 1,   // + stage
+    BB_X_EMPTY = 3,  // + stage
+    BB_Y_FULL = 5,   // + stage
+    BB_Y_EMPTY = 7,  // + stage
+    BB_S_FULL = 9,
+    BB_P_FULL = 10,
+    BB_ACC_DONE = 11,  // the gradient MMAs of a step have read the dS / P operands in TMEM
+    BB_FINAL = 12,
+    BB_COUNT = 13
+};
+
+struct BwdParams {
+    MaskGeom g;
+    int nb, H, mode;
+    const int* ptr;            // row_ptr (dQ pass) or col_ptr (dK/dV pass)
+    const int* idx;            // col_idx or row_idx
+    const unsigned char* flag; // flag or tflag
+    const float* lse;          // [B*H, n] natural log
+    const float* Dv;           // [B*H, n] rowsum(dO * O)
+    __nv_bfloat16* out0;       // dQ, or dK
+    __nv_bfloat16* out1;       // unused, or dV
+    float scale, scale_log2;
+    int* err;
+    unsigned long long timeout_ns;
+};
+
+// Barrier over the 128 gradient threads that also ANDs a predicate across them,
+// so that all four warps take the same abort decision.
+__device__ __forceinline__ bool sync_and_128(bool pred)
+{
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.red.and.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(out)
+        : "r"(static_cast<uint32_t>(pred))
+        : "memory");
+    return out != 0;
+}
+
+template <int D, bool TRANS>
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tmR0, const __grid_constant__ CUtensorMap tmR1,
+               const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY, const BwdParams p)
+{
+    using L = BLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_addr(smem_raw);
+    const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (sbase - raw_addr);
+    const uint32_t sR0 = sbase + L::R0_OFF, sR1 = sbase + L::R1_OFF, sX = sbase + L::X_OFF, sY = sbase + L::Y_OFF;
+    const uint32_t bars = sbase + L::BAR_OFF;
+    auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::BAR_OFF + 8 * BB_COUNT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::BAR_OFF + 8 * BB_COUNT + 4);
+    float* stat = reinterpret_cast<float*>(smem + L::STAT_OFF);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;  // tb: query tile (dQ) or key tile (dK/dV)
+    const int bh = b * p.H + h;
+    const int n = p.g.n;
+    WaitCtl wc{abort_flag, p.err, p.timeout_ns};
+
+    if (threadIdx.x == 0) {
+        *abort_flag = *reinterpret_cast<volatile int*>(p.err) != 0 ? 1 : 0;
+        for (int i = 0; i < BB_COUNT; ++i)
+            mbar_init(bar(i), i == BB_P_FULL ? 128u : 1u);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 5) {
+        tmem_alloc(smem_addr(tmem_slot), BWD_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const bool skip = *abort_flag != 0;
+    const int start = p.ptr[tb];
+    const int len = skip ? 0 : p.ptr[tb + 1] - start;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0 && len > 0) {
+            mbar_arrive_expect_tx(bar(BB_RES_FULL), 2 * L::TILE_BYTES);
+            for (int c = 0; c < L::CHUNKS; ++c) {
+                tma_load_3d(sR0 + c * L::CHUNK_BYTES, &tmR0, bar(BB_RES_FULL), c * 64, tb * TILE, bh);
+                tma_load_3d(sR1 + c * L::CHUNK_BYTES, &tmR1, bar(BB_RES_FULL), c * 64, tb * TILE, bh);
+            }
+            int x_issued = 0, y_issued = 0;
+            for (int j = 0; j < len; ++j) {
+                const int other = p.idx[start + j];
+                const int st = j % L::STAGES;
+                if (j >= L::STAGES && !mbar_wait(bar(BB_X_EMPTY + st), ((j / L::STAGES) - 1) & 1, wc, BSITE_X_EMPTY))
+                    break;
+                mbar_arrive_expect_tx(bar(BB_X_FULL + st), L::TILE_BYTES);
+                for (int c = 0; c < L::CHUNKS; ++c)
+                    tma_load_3d(sX + st * L::TILE_BYTES + c * L::CHUNK_BYTES, &tmX, bar(BB_X_FULL + st), c * 64,
+                                other * TILE, bh);
+                x_issued = j + 1;
+                if (j >= L::STAGES && !mbar_wait(bar(BB_Y_EMPTY + st), ((j / L::STAGES) - 1) & 1, wc, BSITE_Y_EMPTY))
+                    break;
+                mbar_arrive_expect_tx(bar(BB_Y_FULL + st), L::TILE_BYTES);
+                for (int c = 0; c < L::CHUNKS; ++c)
+                    tma_load_3d(sY + st * L::TILE_BYTES + c * L::CHUNK_BYTES, &tmY, bar(BB_Y_FULL + st), c * 64,
+                                other * TILE, bh);
+                y_issued = j + 1;
+            }
+            drain_wait(bar(BB_RES_FULL), 0, p.timeout_ns);
+            for (int j = max(0, x_issued - L::STAGES); j < x_issued; ++j)
+                drain_wait(bar(BB_X_FULL + j % L::STAGES), (j / L::STAGES) & 1, p.timeout_ns);
+            for (int j = max(0, y_issued - L::STAGES); j < y_issued; ++j)
+                drain_wait(bar(BB_Y_FULL + j % L::STAGES), (j / L::STAGES) & 1, p.timeout_ns);
+        }
+    } else if (warp == 5) {
+        // ----------------------------------------------------------------- MMA
+        if (lane == 0 && len > 0) {
+            constexpr uint32_t idesc_nt = idesc_bf16_f32(TILE, TILE, 0, 0);  // A, B K-major
+            constexpr uint32_t idesc_acc = idesc_bf16_f32(TILE, D, 0, 1);    // A from TMEM, B MN-major
+            // D[col] = A(smem tile a) * B(smem tile b)^T over d.
+            auto mma_nt = [&](uint32_t col, uint32_t a, uint32_t b2) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
+                    mma_ss(tmem + col, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b2 + off, 16, 1024),
+                           idesc_nt, kk > 0 ? 1u : 0u);
+                }
+            };
+            // acc[col] += A(TMEM, 128 x 128 bf16 at acol) * B(smem tile b, 128 x d, MN-major).
+            auto mma_acc = [&](uint32_t col, uint32_t acol, uint32_t b2, bool first) {
+#pragma unroll
+                for (int kk = 0; kk < TILE / 16; ++kk)
+                    mma_ts(tmem + col, tmem + acol + kk * 8, smem_desc_sw128(b2 + kk * 2048, L::CHUNK_BYTES, 1024),
+                           idesc_acc, (!first || kk > 0) ? 1u : 0u);
+            };
+            bool ok = mbar_wait(bar(BB_RES_FULL), 0, wc, BSITE_RES);
+            tc_fence_after();
+            for (int j = 0; ok && j < len; ++j) {
+                const int st = j % L::STAGES;
+                if (!(ok = mbar_wait(bar(BB_X_FULL + st), (j / L::STAGES) & 1, wc, BSITE_X_FULL)) ||
+                    !(ok = mbar_wait(bar(BB_Y_FULL + st), (j / L::STAGES) & 1, wc, BSITE_Y_FULL)))
+                    break;
+                // The next S / dP overwrite the TMEM columns that the previous
+                // step's gradient MMAs read as operands; MMAs into different
+                // accumulators are not ordered, so wait for those first.
+                if (j > 0 && !(ok = mbar_wait(bar(BB_ACC_DONE), (j - 1) & 1, wc, BSITE_ACC)))
+                    break;
+                tc_fence_after();
+                const uint32_t x = sX + st * L::TILE_BYTES, y = sY + st * L::TILE_BYTES;
+                mma_nt(COL_S, sR0, x);   // S = Q K^T, or S^T = K Q^T
+                mma_nt(COL_DP, sR1, y);  // dP = dO V^T, or dP^T = V dO^T
+                mma_commit(bar(BB_S_FULL));
+                if (!(ok = mbar_wait(bar(BB_P_FULL), j & 1, wc, BSITE_P_FULL)))
+                    break;
+                tc_fence_after();
+                if (!TRANS) {
+                    mma_acc(COL_ACC0, COL_S, x, j == 0);   // dQ += dS K
+                } else {
+                    mma_acc(COL_ACC1, COL_S, y, j == 0);   // dV += P^T dO
+                    mma_acc(COL_ACC0, COL_DP, x, j == 0);  // dK += dS^T Q
+                }
+                mma_commit(bar(BB_ACC_DONE));
+                mma_commit(bar(BB_X_EMPTY + st));
+                mma_commit(bar(BB_Y_EMPTY + st));
+            }
+            mma_commit(bar(BB_FINAL));
+            drain_wait(bar(BB_FINAL), 0, p.timeout_ns);
+        }
+    } else {
+        // ------------------------------------------------------ gradient warps
+        const int t = threadIdx.x;  // == TMEM lane: query row (dQ) or key row (dK/dV) of the tile
+        const int row = tb * TILE + t;
+        const bool row_valid = row < n;
+        const int rf = row_valid ? row / p.g.s : 0, rp = row_valid ? row % p.g.s : 0;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const bool tail = (n % TILE) != 0;
+        // per-row statistics of a query row (dQ pass)
+        const float row_l2 = (!TRANS && row_valid) ? p.lse[static_cast<size_t>(bh) * n + row] * LOG2E : 0.f;
+        const float row_d = (!TRANS && row_valid) ? p.Dv[static_cast<size_t>(bh) * n + row] : 0.f;
+        bool ok = true;
+        for (int j = 0; j < len; ++j) {
+            const int other = p.idx[start + j];  // key tile (dQ) or query tile (dK/dV)
+            const bool partial = p.flag[start + j] != RA_TILE_FULL;
+            float* st_l2 = stat + (j & 1) * 2 * TILE;
+            float* st_d = st_l2 + TILE;
+            if (TRANS) {
+                // statistics of the query tile's 128 columns; columns >= n get
+                // L = +inf so their P is exactly 0
+                const int q = other * TILE + t;
+                st_l2[t] = q < n ? p.lse[static_cast<size_t>(bh) * n + q] * LOG2E : INFINITY;
+                st_d[t] = q < n ? p.Dv[static_cast<size_t>(bh) * n + q] : 0.f;
+            }
+            uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
+            const bool use_family = p.mode == RA_MODE_TOKEN_EXACT && partial;
+            const bool masked = use_family || (!TRANS && tail && other == p.nb - 1);
+            if (masked) {
+                if (use_family && row_valid) {
+                    if (!TRANS)
+                        row_keep_mask(p.g, rf, rp, other * TILE, mk[0], mk[1], mk[2], mk[3]);
+                    else
+                        col_keep_mask(p.g, rf, rp, other * TILE, mk[0], mk[1], mk[2], mk[3]);
+                } else if (!TRANS) {
+                    const int valid_cols = min(TILE, n - other * TILE);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int v = valid_cols - 32 * c;
+                        mk[c] = v >= 32 ? 0xFFFFFFFFu : (v <= 0 ? 0u : ((1u << v) - 1u));
+                    }
+                }
+            }
+            ok = mbar_wait(bar(BB_S_FULL), j & 1, wc, BSITE_S_FULL);
+            // one decision for all 128 threads; also publishes the staged statistics
+            ok = TRANS ? sync_and_128(ok) : __all_sync(0xFFFFFFFFu, ok);
+            if (!ok)
+                break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t sv[32], dv[32];
+                tmem_ld32(lane_base + COL_S + c * 32, sv);
+                tmem_ld32(lane_base + COL_DP + c * 32, dv);
+                tmem_wait_ld();
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float pe[2], ds[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int col = c * 32 + e + u;
+                        const bool keep = !masked || ((mk[c] >> (e + u)) & 1u);
+                        const float l2 = TRANS ? st_l2[col] : row_l2;
+                        const float dd = TRANS ? st_d[col] : row_d;
+                        const float x = fmaf(__uint_as_float(sv[e + u]), p.scale_log2, -l2);
+                        pe[u] = keep ? fast_exp2(x) : 0.f;
+                        ds[u] = pe[u] * (__uint_as_float(dv[e + u]) - dd);
+                    }
+                    pk[e >> 1] = pack_bf16(pe[0], pe[1]);
+                    dk[e >> 1] = pack_bf16(ds[0], ds[1]);
+                }
+                // Written over columns already read (chunk c goes to columns 16 c .. 16 c + 15).
+                if (!TRANS) {
+                    tmem_st16(lane_base + COL_S + c * 16, dk);   // dS for dQ += dS K
+                } else {
+                    tmem_st16(lane_base + COL_S + c * 16, pk);   // P^T for dV += P^T dO
+                    tmem_st16(lane_base + COL_DP + c * 16, dk);  // dS^T for dK += dS^T Q
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(BB_P_FULL));
+        }
+        // ------------------------------------------------------------ epilogue
+        if (len > 0 && ok)
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(BB_FINAL), 0, wc, BSITE_FINAL));
+        tc_fence_after();
+        if (ok && !*abort_flag && row_valid) {
+#pragma unroll 1
+            for (int which = 0; which < (TRANS ? 2 : 1); ++which) {
+                __nv_bfloat16* dst_row = (which == 0 ? p.out0 : p.out1) + (static_cast<size_t>(bh) * n + row) * D;
+                const float mul = which == 0 ? p.scale : 1.f;  // dQ, dK carry the softmax scale; dV does not
+                const uint32_t col0 = which == 0 ? COL_ACC0 : COL_ACC1;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    if (len > 0) {
+                        tmem_ld32(lane_base + col0 + c * 32, o);
+                        tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            o[e] = 0u;
+                    }
+                    uint4 v[4];
+                    uint32_t* w = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2)
+                        w[e >> 1] = pack_bf16(__uint_as_float(o[e]) * mul, __uint_as_float(o[e + 1]) * mul);
+                    uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        dst[u] = v[u];
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5) {
+        __syncwarp();
+        tmem_dealloc(tmem, BWD_TMEM_COLS);
+    }
+}
+
+// D[r] = <dO[r], O[r]> over d, one warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dot_kernel(const __nv_bfloat16* __restrict__ O,
+                                                      const __nv_bfloat16* __restrict__ dO, float* __restrict__ Dv,
+                                                      long long rows)
+{
+    const long long warp_id = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+    for (long long r = warp_id; r < rows; r += nwarps) {
+        float acc = 0.f;
+#pragma unroll
+        for (int k = lane * 2; k < D; k += 64) {
+            const __nv_bfloat162 o = *reinterpret_cast<const __nv_bfloat162*>(O + r * D + k);
+            const __nv_bfloat162 g = *reinterpret_cast<const __nv_bfloat162*>(dO + r * D + k);
+            acc = fmaf(__low2float(o), __low2float(g), acc);
+            acc = fmaf(__high2float(o), __high2float(g), acc);
+        }
+        for (int off = 16; off > 0; off >>= 1)
+            acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+        if (lane == 0)
+            Dv[r] = acc;
+    }
+}
+
+template <int D, bool TRANS>
+ra_status launch_bwd(const CUtensorMap& r0, const CUtensorMap& r1, const CUtensorMap& x, const CUtensorMap& y,
+                     const BwdParams& p, int B, cudaStream_t cs)
+{
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(bwd_kernel<D, TRANS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        BLayout<D>::SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess)
+        return cuda_fail(attr_err, "cudaFuncSetAttribute(bwd_kernel)");
+    dim3 grid(p.nb, p.H, B);
+    bwd_kernel<D, TRANS><<<grid, BWD_THREADS, BLayout<D>::SMEM_BYTES, cs>>>(r0, r1, x, y, p);
+    return cuda_fail(cudaGetLastError(), "bwd_kernel launch");
+}
+
+template <int D>
+ra_status run_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* lse,
+                  void* dQ, void* dK, void* dV, float* Dws, int B, int H, const ra_mask* m, float scale, int mode,
+                  cudaStream_t cs)
+{
+    const int BH = B * H, n = m->geom.n;
+    const long long rows = static_cast<long long>(BH) * n;
+    const int dot_blocks = static_cast<int>(std::min<long long>((rows + 7) / 8, 148LL * 16));
+    bwd_dot_kernel<D><<<dot_blocks, 256, 0, cs>>>(static_cast<const __nv_bfloat16*>(O),
+                                                  static_cast<const __nv_bfloat16*>(dO), Dws, rows);
+    ra_status st = cuda_fail(cudaGetLastError(), "bwd_dot_kernel launch");
+    if (st != RA_OK)
+        return st;
+    CUtensorMap mq, mk, mv, mdo;
+    if ((st = make_map(&mq, Q, BH, n, D, TILE)) != RA_OK || (st = make_map(&mk, K, BH, n, D, TILE)) != RA_OK ||
+        (st = make_map(&mv, V, BH, n, D, TILE)) != RA_OK || (st = make_map(&mdo, dO, BH, n, D, TILE)) != RA_OK)
+        return st;
+    BwdParams p;
+    std::memset(&p, 0, sizeof p);
+    p.g = m->geom;
+    p.nb = m->nb;
+    p.H = H;
+    p.mode = mode;
+    p.lse = lse;
+    p.Dv = Dws;
+    p.scale = scale;
+    p.scale_log2 = scale * LOG2E;
+    p.timeout_ns = wait_timeout_ns();
+    if ((st = device_error_word(&p.err)) != RA_OK)
+        return st;
+    // dQ: query tiles over the block-CSR rows; resident Q, dO; ring K, V
+    p.ptr = m->row_ptr;
+    p.idx = m->col_idx;
+    p.flag = m->flag;
+    p.out0 = static_cast<__nv_bfloat16*>(dQ);
+    p.out1 = nullptr;
+    if ((st = launch_bwd<D, false>(mq, mdo, mk, mv, p, B, cs)) != RA_OK)
+        return st;
+    // dK, dV: key tiles over the transposed block-CSR; resident K, V; ring Q, dO
+    p.ptr = m->col_ptr;
+    p.idx = m->row_idx;
+    p.flag = m->tflag;
+    p.out0 = static_cast<__nv_bfloat16*>(dK);
+    p.out1 = static_cast<__nv_bfloat16*>(dV);
+    return launch_bwd<D, true>(mk, mv, mq, mdo, p, B, cs);
+}
+
+}  // namespace
+}  // namespace ra
+
+using namespace ra;
+
+extern "C" ra_status ra_attention_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                                      const float* lse, void* dQ, void* dK, void* dV, float* D_workspace, int B,
+                                      int H, int d, const ra_mask* m, float scale, int mode, ra_stream stream)
+{
+    const void* ptrs[9] = {Q, K, V, O, dO, dQ, dK, dV, nullptr};
+    for (int i = 0; i < 8; ++i) {
+        if (!ptrs[i])
+            return fail(RA_ERR_INVALID_ARG, "NULL tensor pointer");
+        if (!aligned16(ptrs[i]))
+            return fail(RA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+    }
+    if (!lse || !D_workspace)
+        return fail(RA_ERR_INVALID_ARG, "NULL lse or workspace");
+    if (!m)
+        return fail(RA_ERR_INVALID_ARG, "NULL mask");
+    if (B < 1 || H < 1 || B > 65535 || H > 65535)
+        return fail(RA_ERR_INVALID_ARG, "B and H must be in [1, 65535] (B=%d, H=%d)", B, H);
+    if (d != 64 && d != 128)
+        return fail(RA_ERR_UNSUPPORTED, "head dim %d is not supported (64 or 128)", d);
+    if (mode != RA_MODE_TOKEN_EXACT && mode != RA_MODE_BLOCK)
+        return fail(RA_ERR_INVALID_ARG, "unknown mode %d", mode);
+    if (!(scale > 0.f) || !std::isfinite(scale))
+        return fail(RA_ERR_INVALID_ARG, "scale must be finite and > 0");
+    if (m->nnz == 0 || !m->col_ptr)
+        return fail(RA_ERR_INVALID_ARG, "mask has no kept tile");
+    int dev = 0;
+    RA_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev != m->device)
+        return fail(RA_ERR_INVALID_ARG, "mask was built on device %d, current device is %d", m->device, dev);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    return d == 64 ? run_bwd<64>(Q, K, V, O, dO, lse, dQ, dK, dV, D_workspace, B, H, m, scale, mode, cs)
+                   : run_bwd<128>(Q, K, V, O, dO, lse, dQ, dK, dV, D_workspace, B, H, m, scale, mode, cs);
+}

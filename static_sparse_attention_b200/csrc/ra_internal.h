@@ -1,5 +1,6 @@
 // ra_internal.h -- state and helpers shared by the library's translation units.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -18,6 +19,11 @@ struct ra_mask {
     int* col_idx;          // [nnz]
     int* count;            // [nnz]
     unsigned char* flag;   // [nnz]
+    // Transposed block-CSR (per key tile, the query tiles that keep it), for the
+    // backward pass: col_ptr [nb + 1], row_idx [nnz] ascending, tflag [nnz].
+    int* col_ptr;
+    int* row_idx;
+    unsigned char* tflag;
 };
 
 namespace ra {
@@ -30,6 +36,28 @@ ra_status cuda_fail(cudaError_t e, const char* what);
 
 // Limit of every bounded device wait, in ns.
 unsigned long long wait_timeout_ns();
+
+// TMA map of a [B*H, n, d] bf16 tensor as a 3D tensor (d, n, B*H), boxes of
+// box_rows rows x 64 columns with 128-byte swizzle; rows beyond n read as zero.
+ra_status make_map(CUtensorMap* map, const void* base, int BH, int n, int d, int box_rows);
+
+// The same for the first `rows` rows of each head of a [B*H, head_rows, d]
+// tensor (rows <= head_rows): rows beyond `rows` read as zero.
+ra_status make_map_rows(CUtensorMap* map, const void* base, int BH, int rows, int head_rows, int d, int box_rows);
+
+// Forward attention of nq query rows per head over the first nk key rows of
+// each head of K and V ([B*H, k_head_rows, d]), walking a caller-supplied
+// block-CSR over nbq query tiles whose key tiles are all treated as FULL
+// (keys >= nk are masked).  Block mode, no family mask: for masks that keep
+// every listed key, such as the window held by the SWC key/value cache.
+ra_status attention_fwd_rect(const void* Q, const void* K, const void* V, void* O, int B, int H, int d, int nq,
+                             int nk, int k_head_rows, const int* row_ptr, const int* col_idx,
+                             const unsigned char* flag, int nbq, float scale, float* lse, cudaStream_t stream);
+
+// Device address of the forward / backward kernels' error word on the current device.
+ra_status device_error_word(int** out);
+
+inline bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
 }  // namespace ra
 

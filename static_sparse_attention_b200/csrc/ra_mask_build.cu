@@ -198,14 +198,66 @@ __global__ void init_totals_kernel(BuildTotals* tot)
     tot->row_max = 0;
 }
 
+// Kept query tiles per key tile (a column of the tile-count matrix).
+__global__ void __launch_bounds__(128) col_count_kernel(const int* __restrict__ counts, int nb,
+                                                        int* __restrict__ col_tiles)
+{
+    __shared__ int part[4];
+    const int kb = blockIdx.x, t = threadIdx.x;
+    int c = 0;
+    for (int qb = t; qb < nb; qb += TILE)
+        c += counts[static_cast<size_t>(qb) * nb + kb] > 0;
+    c = __reduce_add_sync(0xFFFFFFFFu, c);
+    if ((t & 31) == 0)
+        part[t >> 5] = c;
+    __syncthreads();
+    if (t == 0)
+        col_tiles[kb] = part[0] + part[1] + part[2] + part[3];
+}
+
+// Kept query tiles of each key tile in ascending order, with the tile's flag.
+__global__ void __launch_bounds__(128) col_compact_kernel(const int* __restrict__ counts, int nb,
+                                                          const int* __restrict__ col_ptr, int* __restrict__ row_idx,
+                                                          unsigned char* __restrict__ tflag)
+{
+    __shared__ int warp_tot[4];
+    const int kb = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    int out = col_ptr[kb];
+    for (int qb0 = 0; qb0 < nb; qb0 += TILE) {
+        const int qb = qb0 + t;
+        const int c = (qb < nb) ? counts[static_cast<size_t>(qb) * nb + kb] : 0;
+        const bool keep = c > 0;
+        const unsigned ballot = __ballot_sync(0xFFFFFFFFu, keep);
+        const int before = __popc(ballot & ((1u << lane) - 1u));
+        if (lane == 0)
+            warp_tot[warp] = __popc(ballot);
+        __syncthreads();
+        int warp_off = 0, chunk = 0;
+        for (int w = 0; w < 4; ++w) {
+            warp_off += (w < warp) ? warp_tot[w] : 0;
+            chunk += warp_tot[w];
+        }
+        if (keep) {
+            const int pos = out + warp_off + before;
+            row_idx[pos] = qb;
+            tflag[pos] = (c == TILE * TILE) ? RA_TILE_FULL : RA_TILE_PARTIAL;
+        }
+        out += chunk;
+        __syncthreads();
+    }
+}
+
 void free_mask_arrays(ra_mask* m)
 {
     cudaFree(m->row_ptr);
     cudaFree(m->col_idx);
     cudaFree(m->count);
     cudaFree(m->flag);
-    m->row_ptr = m->col_idx = m->count = nullptr;
-    m->flag = nullptr;
+    cudaFree(m->col_ptr);
+    cudaFree(m->row_idx);
+    cudaFree(m->tflag);
+    m->row_ptr = m->col_idx = m->count = m->col_ptr = m->row_idx = nullptr;
+    m->flag = m->tflag = nullptr;
 }
 
 struct Scratch {
@@ -335,6 +387,22 @@ extern "C" ra_status ra_build_mask(int family, int f, int s, const ra_mask_param
         compact_kernel<<<nb, TILE, 0, cs>>>(sc.counts, nb, m->row_ptr, m->col_idx, m->count, m->flag);
         if ((e = cudaGetLastError()) != cudaSuccess)
             return bail(e, "compact_kernel launch");
+        // transposed block-CSR for the backward pass (same nnz)
+        if ((e = cudaMalloc(&m->col_ptr, sizeof(int) * (nb + 1))) != cudaSuccess)
+            return bail(e, "col_ptr");
+        if ((e = cudaMalloc(&m->row_idx, sizeof(int) * nnz)) != cudaSuccess)
+            return bail(e, "row_idx");
+        if ((e = cudaMalloc(&m->tflag, nnz)) != cudaSuccess)
+            return bail(e, "tflag");
+        col_count_kernel<<<nb, TILE, 0, cs>>>(sc.counts, nb, sc.row_tiles);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return bail(e, "col_count_kernel launch");
+        row_scan_kernel<<<1, 1024, 0, cs>>>(sc.row_tiles, nb, m->col_ptr);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return bail(e, "column scan launch");
+        col_compact_kernel<<<nb, TILE, 0, cs>>>(sc.counts, nb, m->col_ptr, m->row_idx, m->tflag);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return bail(e, "col_compact_kernel launch");
     }
     // The scratch arrays are released by ~Scratch; cudaFree waits for the kernels.
     if ((e = cudaStreamSynchronize(cs)) != cudaSuccess)
@@ -480,6 +548,22 @@ extern "C" ra_status ra_build_mask_noalloc(int family, int f, int s, const ra_ma
     if (nnz > 0) {
         compact_kernel<<<nb, TILE, 0, cs>>>(counts, nb, row_ptr, col_idx, count, flag);
         RA_CUDA_TRY(cudaGetLastError());
+    }
+    return RA_OK;
+}
+
+extern "C" ra_status ra_mask_copy_transpose_to_host(const ra_mask* m, int* col_ptr, int* row_idx,
+                                                    unsigned char* tflag)
+{
+    if (!m)
+        return fail(RA_ERR_INVALID_ARG, "NULL mask");
+    if (col_ptr)
+        RA_CUDA_TRY(cudaMemcpy(col_ptr, m->col_ptr, sizeof(int) * (m->nb + 1), cudaMemcpyDeviceToHost));
+    if (m->nnz > 0) {
+        if (row_idx)
+            RA_CUDA_TRY(cudaMemcpy(row_idx, m->row_idx, sizeof(int) * m->nnz, cudaMemcpyDeviceToHost));
+        if (tflag)
+            RA_CUDA_TRY(cudaMemcpy(tflag, m->tflag, m->nnz, cudaMemcpyDeviceToHost));
     }
     return RA_OK;
 }

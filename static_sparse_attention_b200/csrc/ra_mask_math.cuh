@@ -156,4 +156,57 @@ __device__ __forceinline__ void row_keep_mask(const MaskGeom& g, int qi, int qk,
     });
 }
 
+// The same for a key column: emit(a, b) for every maximal run of queries
+// [a, b] inside [c0, c1] that keep key (frame kj, position kk).  The radial
+// mask (|i-j|, |k-l|), the 3D window (|dt|, |dh|, |dw|), the dense mask and the
+// global tokens are symmetric, so a key's queries are its own row's keys; the
+// causal sliding window keeps query frames kj .. kj + W - 1.
+template <class Emit>
+__device__ __forceinline__ void for_each_kept_query_run(const MaskGeom& g, int kj, int kk, int c0, int c1,
+                                                        Emit&& emit)
+{
+    if (g.family != FAM_SWC) {
+        for_each_kept_run(g, kj, kk, c0, c1, emit);
+        return;
+    }
+    if (g.sink > 0) {
+        if (kj * g.s + kk < g.sink) {
+            emit(c0, c1);
+            return;
+        }
+        if (c0 < g.sink) {
+            emit(c0, min(c1, g.sink - 1));
+            c0 = g.sink;
+            if (c0 > c1)
+                return;
+        }
+    }
+    const int s = g.s;
+    const int lo = max(c0 / s, kj), hi = min(c1 / s, kj + g.window_frames - 1);
+    if (lo <= hi)
+        emit(max(c0, lo * s), min(c1, hi * s + s - 1));
+}
+
+// 128-bit keep mask of a key column over the query rows [c0, c0 + 127].
+__device__ __forceinline__ void col_keep_mask(const MaskGeom& g, int kj, int kk, int c0, uint32_t& m0, uint32_t& m1,
+                                              uint32_t& m2, uint32_t& m3)
+{
+    m0 = m1 = m2 = m3 = 0u;
+    const int c1 = min(c0 + TILE - 1, g.n - 1);
+    for_each_kept_query_run(g, kj, kk, c0, c1, [&](int a, int b) {
+        const int lo = a - c0, hi = b - c0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int l = max(lo, 32 * w), h = min(hi, 32 * w + 31);
+            if (l <= h) {
+                const uint32_t bits = bit_range(l - 32 * w, h - 32 * w);
+                if (w == 0) m0 |= bits;
+                else if (w == 1) m1 |= bits;
+                else if (w == 2) m2 |= bits;
+                else m3 |= bits;
+            }
+        }
+    });
+}
+
 }  // namespace ra

@@ -84,7 +84,7 @@ struct WaitCtl {
     uint64_t timeout_ns;
 };
 
-__device__ __noinline__ void report_timeout(const WaitCtl& w, int site)
+static __device__ __noinline__ void report_timeout(const WaitCtl& w, int site)
 {
     *w.abort_flag = 1;
     if (atomicCAS(w.err_word, 0, 5 /* RA_ERR_DEVICE_TIMEOUT */) == 0) {
@@ -223,6 +223,33 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
         "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
+}
+
+// ----------------------------------------------------------------- misc
+#include <cuda_bf16.h>
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Wait without the CTA abort flag: used only to drain in-flight copies and
+// MMAs before the CTA releases its memory.
+static __device__ bool drain_wait(uint32_t bar, uint32_t parity, unsigned long long timeout_ns)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > timeout_ns)
+            return false;
+    }
+    return true;
 }
 
 // ----------------------------------------------------------- descriptors

@@ -96,6 +96,42 @@ def test_attention_rejects_bad_arguments(ra):
                                     None) == ra.RA_ERR_INVALID_ARG
 
 
+def test_backward_rejects_bad_arguments(ra):
+    fake = ctypes.c_void_p(0x10000)  # never dereferenced: validation fails first
+    args = dict(Q=0x10000, K=0x20000, V=0x30000, O=0x40000, dO=0x50000, lse=0x60000, dQ=0x70000, dK=0x80000,
+                dV=0x90000, ws=0xA0000, B=1, H=1, d=128, m=fake, scale=0.1, mode=1)
+
+    def call(**kw):
+        a = {**args, **kw}
+        return ra.ra_attention_bwd(a["Q"], a["K"], a["V"], a["O"], a["dO"], a["lse"], a["dQ"], a["dK"], a["dV"],
+                                   a["ws"], a["B"], a["H"], a["d"], a["m"], a["scale"], a["mode"], None)
+
+    assert call(dO=None) == ra.RA_ERR_INVALID_ARG
+    assert call(dV=0x90004) == ra.RA_ERR_INVALID_ARG         # not 16-byte aligned
+    assert call(lse=None) == ra.RA_ERR_INVALID_ARG
+    assert call(ws=None) == ra.RA_ERR_INVALID_ARG
+    assert call(m=None) == ra.RA_ERR_INVALID_ARG
+    assert call(B=0) == ra.RA_ERR_INVALID_ARG
+    assert call(d=256) == ra.RA_ERR_UNSUPPORTED
+    assert call(mode=3) == ra.RA_ERR_INVALID_ARG
+    assert call(scale=-1.0) == ra.RA_ERR_INVALID_ARG
+
+
+def test_swc_cache_rejects_bad_arguments(ra):
+    h = ctypes.c_void_p()
+    assert ra.ra_swc_cache_create(0, 1, 128, 100, 4, ctypes.byref(h)) == ra.RA_ERR_INVALID_ARG
+    assert ra.ra_swc_cache_create(1, 1, 96, 100, 4, ctypes.byref(h)) == ra.RA_ERR_UNSUPPORTED
+    assert ra.ra_swc_cache_create(1, 1, 128, 0, 4, ctypes.byref(h)) == ra.RA_ERR_INVALID_ARG
+    assert ra.ra_swc_cache_create(1, 1, 128, 100, 0, ctypes.byref(h)) == ra.RA_ERR_INVALID_ARG
+    assert ra.ra_swc_cache_create(1, 1, 128, 100, 4, None) == ra.RA_ERR_INVALID_ARG
+    assert ra.ra_swc_cache_create(1, 1, 64, 1 << 20, 4096, ctypes.byref(h)) == ra.RA_ERR_UNSUPPORTED
+    assert ra.ra_swc_cache_step(None, None, None, None, None, 0.1, None, None) == ra.RA_ERR_INVALID_ARG
+    assert ra.ra_swc_cache_info(None, None, None) == ra.RA_ERR_INVALID_ARG
+    assert ra.ra_swc_cache_reset(None) == ra.RA_ERR_INVALID_ARG
+    assert ra.ra_swc_cache_copy_rings_to_host(None, None, None) == ra.RA_ERR_INVALID_ARG
+    ra.ra_swc_cache_free(None)
+
+
 def test_timeout_settings_are_range_checked(ra):
     assert ra.ra_set_wait_timeout_ns(10) == ra.RA_ERR_INVALID_ARG
     assert ra.ra_set_wait_timeout_ns(4_000_000_000) == ra.RA_OK
