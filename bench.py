@@ -39,6 +39,7 @@ import synth  # noqa: E402
 METRIC = "radial sparse-attn fwd ms & effective TFLOP/s (bf16, % of TC peak), 1 B200"
 METRIC_BWD = "radial sparse-attn bwd ms & effective TFLOP/s (bf16, % of TC peak), 1 B200"
 METRIC_STREAM = "SWC streaming step (KV ring cache) ms per frame & effective TFLOP/s (bf16), 1 B200"
+METRIC_POLICY = "dense-first schedule: attention ms per denoising step & effective TFLOP/s (bf16), 1 B200"
 L2_BYTES = 126 * 1024 * 1024
 ATTN_SOURCES = {
     "fwd": ["static_sparse_attention_b200/csrc/ra_attention.cu", "static_sparse_attention_b200/csrc/ra_sm100.cuh",
@@ -61,8 +62,13 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (small profiling cases)")
-    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd", "stream"],
-                    help="time the forward (default), the backward, or the streaming SWC step")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd", "stream", "policy"],
+                    help="time the forward (default), the backward, the streaming SWC step, or a whole "
+                         "dense-first denoising schedule of forward calls")
+    ap.add_argument("--policy-steps", type=int, default=50, help="denoising steps of the policy schedule")
+    ap.add_argument("--policy-blocks", type=int, default=40, help="attention blocks per denoising step")
+    ap.add_argument("--dense-steps", type=int, default=12, help="first steps that run every block dense")
+    ap.add_argument("--dense-blocks", type=int, default=2, help="first blocks that run dense at every step")
     return ap.parse_args()
 
 
@@ -253,13 +259,14 @@ def run_reference(args, c, mask):
                                                         target_s=per_step)
         else:
             v, threads, desc = cpu_oracle_sample(args.workload, c["masks"][args.mask], args.mode, c,
-                                                 target_s=per_step, kind=args.pass_)
+                                                 target_s=per_step, kind="bwd" if args.pass_ == "bwd" else "fwd")
         if i >= args.warmup:
             vals.append(v)
             descs.append(desc)
     value = float(np.median(vals))
     line = {
-        "impl": "reference", "metric": {"fwd": METRIC, "bwd": METRIC_BWD, "stream": METRIC_STREAM}[args.pass_],
+        "impl": "reference",
+        "metric": {"fwd": METRIC, "bwd": METRIC_BWD, "stream": METRIC_STREAM, "policy": METRIC_POLICY}[args.pass_],
         "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -446,6 +453,103 @@ def run_stream(args, c, mask, world, rank, dev):
     print(json.dumps(line), flush=True)
 
 
+def run_policy(args, c, mask, world, rank, dev):
+    """A whole denoising schedule of forward calls: at step t and block l the
+    dense mask when t < dense_steps or l < dense_blocks, else the workload's
+    sparse mask (the dense warm-up of the first steps and the dense first DiT
+    blocks).  One timed step = one denoising step (policy_blocks calls); the
+    schedule runs policy_steps of them, so --steps / --warmup are not used."""
+    import torch
+    import torch.distributed as dist
+
+    import static_sparse_attention_b200 as ra
+
+    B, H, d = c["B"], c["H"], c["d"]
+    n = c["f"] * c["s"]
+    shape = (B, H, n, d)
+    seed = synth.config_seed(args.workload)
+    host = [synth.normal_bf16(seed, tid, shape) for tid in rank_tensor_ids(rank)]
+    q, k, v = (torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).to(f"cuda:{dev}") for h in host)
+    o = torch.empty_like(q)
+    sparse = ra.build_mask(mask, c["f"], c["s"], c["grid"])
+    dense = ra.build_mask(dict(family="dense"), c["f"], c["s"])
+    policy = ra.DenseFirstPolicy(sparse, dense, dense_steps=args.dense_steps, dense_blocks=args.dense_blocks)
+    scale = 1.0 / math.sqrt(d)
+    stream = torch.cuda.current_stream()
+    T, L = args.policy_steps, args.policy_blocks
+    f_sparse = flops_per_call(sparse.info, c, args.mode)
+    f_dense = flops_per_call(dense.info, c, "block")
+
+    def call(m):
+        ra.attention_fwd(q, k, v, m, scale=scale, mode=args.mode if m is sparse else "block", out=o, stream=stream)
+
+    # per-call times of each mask, for the all-dense and all-sparse reference points
+    per_call = {}
+    for name, m in (("sparse", sparse), ("dense", dense)):
+        for _ in range(2):
+            call(m)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(3):
+            call(m)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        per_call[name] = e0.elapsed_time(e1) / 3
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    flop = 0.0
+    n_dense = 0
+    with ClockSampler(physical_gpu(dev)) as clk:
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for t in range(T):
+            for l in range(L):
+                m = policy.mask(t, l)
+                n_dense += m is dense
+                flop += f_dense if m is dense else f_sparse
+                call(m)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if ra.device_status() != ra.RA_OK:
+        raise SystemExit("device status error after the timed region")
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world, f"cuda:{dev}")
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    calls = T * L
+    all_dense_ms = calls * per_call["dense"]
+    burst, sustained, _, peak_src = measured_peaks()
+    achieved = flop / (total_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC_POLICY, "value": flop * world / (total_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": T, "warmup": 2, "ms_per_step": total_ms / T, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": workload_desc(args.workload, mask, args.mode, c),
+            "pass": "policy", "policy": f"dense when step < {args.dense_steps} or block < {args.dense_blocks}, "
+                                        f"else {mask['family']}",
+            "denoising_steps": T, "blocks_per_step": L, "calls": calls, "dense_calls": n_dense,
+            "l2": "inputs larger than L2 (Q+K+V+O per call)",
+        },
+        "schedule_ms": total_ms, "all_dense_schedule_ms_from_per_call": all_dense_ms,
+        "speedup_vs_all_dense": all_dense_ms / total_ms,
+        "per_call_ms": per_call,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
+                     "frac": achieved / sustained, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 sustained (a schedule of many calls)",
+                     "kernel": "attn_fwd_kernel<%d> (sparse and dense calls)" % d, "flop_per_launch": flop / calls},
+        "clocks": clk.summary(),
+        "gpu_launches": calls,
+        "e2e": None,
+        "cpu_baseline": None,
+        "pages_context": "first 2 DiT blocks and first 12 denoising steps dense (Radial Attention, sec. 6)",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     c = dict(synth.CONFIGS[args.workload])
@@ -464,6 +568,9 @@ def main():
     world, rank, dev = init_ranks()
     if args.pass_ == "stream":
         run_stream(args, c, mask, world, rank, dev)
+        return
+    if args.pass_ == "policy":
+        run_policy(args, c, mask, world, rank, dev)
         return
 
     B, H, d = c["B"], c["H"], c["d"]

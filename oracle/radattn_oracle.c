@@ -478,7 +478,8 @@ void oracle_attention_bwd_query_rows(const void* Q, const void* K, const void* V
 
 /*
  * dK and dV of listed key rows of one (batch, head) slice (Q, K, V, dO: [n, d]):
- * first lse_i and D_i of every query row, then for each listed key j
+ * first lse_i and D_i of every query row that keeps at least one listed key,
+ * then for each listed key j
  *   dK_j = scale sum_i P_ij (<dO_i, V_j> - D_i) Q_i,   dV_j = sum_i P_ij dO_i
  * over the queries i whose row keeps j.  O(n * keys * d) for the statistics,
  * O(n * d) per listed key.  tile_flags: the whole nb x nb table (block mode).
@@ -499,6 +500,12 @@ void oracle_attention_bwd_key_rows(const void* Q, const void* K, const void* V, 
         double* o = (double*)malloc(sizeof(double) * (size_t)d);
 #pragma omp for schedule(dynamic, 16)
         for (long long i = 0; i < n; i++) {
+            int needed = 0;
+            for (long long r = 0; r < nkeys && !needed; r++)
+                needed = mode == OR_TOKEN_EXACT ? oracle_kept(sp, i, key_idx[r])
+                                                : tile_flags[(i / OR_TILE) * nb + key_idx[r] / OR_TILE] != 0;
+            if (!needed)
+                continue; /* row i keeps none of the listed keys: its statistics are not used */
             const unsigned char* flags = mode == OR_TOKEN_EXACT ? NULL : tile_flags + (i / OR_TILE) * nb;
             long long m = or_row_scores(Q, K, dtype, n, d, sp, mode, scale, i, flags, i * d, 0, idx, x, &lse[i]);
             for (int c = 0; c < d; c++)

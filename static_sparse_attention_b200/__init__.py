@@ -304,6 +304,32 @@ class SwcCache:
             pass
 
 
+class DenseFirstPolicy:
+    """Which mask a denoising step uses in each attention block: dense for the
+    first `dense_steps` steps (warm-up) and, at every step, for the first
+    `dense_blocks` blocks; the sparse mask elsewhere ("Radial Attention",
+    sec. 6: the first 2 DiT blocks and the first 12 denoising steps stay dense)."""
+
+    def __init__(self, sparse: Mask, dense: Mask, dense_steps: int = 12, dense_blocks: int = 2):
+        if dense_steps < 0 or dense_blocks < 0:
+            raise ValueError("dense_steps and dense_blocks must be >= 0")
+        if sparse.n != dense.n:
+            raise ValueError("both masks must cover the same tokens")
+        self.sparse, self.dense = sparse, dense
+        self.dense_steps, self.dense_blocks = dense_steps, dense_blocks
+
+    def is_dense(self, step: int, block: int) -> bool:
+        return step < self.dense_steps or block < self.dense_blocks
+
+    def mask(self, step: int, block: int) -> Mask:
+        return self.dense if self.is_dense(step, block) else self.sparse
+
+    def dense_calls(self, steps: int, blocks: int) -> int:
+        """Dense calls in a schedule of `steps` x `blocks` attention calls."""
+        warm = min(self.dense_steps, steps)
+        return warm * blocks + (steps - warm) * min(self.dense_blocks, blocks)
+
+
 def device_status(stream=None) -> int:
     """Synchronise and read (then clear) the device error word; returns the status code."""
     return ra_get_device_status(_stream_handle(stream))

@@ -7,17 +7,21 @@
 //   dQ = scale dS K,   dK = scale dS^T Q,   dV = P^T dO.
 // Deterministic: no atomics, each output tile is owned by one CTA.
 //
-//   bwd_dot_kernel   D = rowsum(dO * O) (fp32), one warp per row.
-//   bwd_kernel<D, false>  one CTA per query tile, walking its block-CSR row:
+//   bwd_dot_kernel         D = rowsum(dO * O) (fp32), one warp per row.
+//   bwd_kernel<D, false>   one CTA per query tile, walking its block-CSR row:
 //       S = Q K^T and dP = dO V^T (tcgen05.mma into TMEM), dS (registers,
 //       bf16 back into TMEM), dQ += dS K (A = dS from TMEM).
-//   bwd_kernel<D, true>   one CTA per key tile, walking the transposed CSR:
+//   bwd_kernel<D, true>    one CTA per key tile, walking the transposed CSR:
 //       S^T = K Q^T and dP^T = V dO^T, P^T and dS^T (bf16 into TMEM),
 //       dV += P^T dO and dK += dS^T Q.
-// Both recompute P from L instead of storing it.  192 threads: warps 0-3 own
-// one tile row each per thread (TMEM lane = row), warp 4 issues the TMA loads
-// (two resident tiles, two 2-stage rings), warp 5 allocates TMEM and issues
-// the MMAs.  TMEM columns: S at 0, dP at 128, the accumulators at 256 and 384.
+// Both recompute P from L instead of storing it.  The walked tiles are taken
+// in 64-row halves ("steps"): the MMAs of step g run while the gradient warps
+// turn step g-1's S and dP into dS, with two TMEM buffers for S and dP.
+// 192 threads: warps 0-3 own one resident row each per thread (TMEM lane =
+// row), warp 4 issues the TMA loads (two resident 128-row tiles, two rings of
+// 64-row halves), warp 5 allocates TMEM and issues the MMAs.
+// TMEM columns: S buffers at 0 and 64, dP buffers at 128 and 192, the
+// accumulators at 256 (dQ or dK) and 384 (dV).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -33,40 +37,49 @@ namespace ra {
 namespace {
 
 constexpr int BWD_THREADS = 192;
+constexpr int HALF = 64;
 constexpr uint32_t BWD_TMEM_COLS = 512;
-constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC0 = 256, COL_ACC1 = 384;
+constexpr uint32_t COL_ACC0 = 256, COL_ACC1 = 384;
 constexpr float LOG2E = 1.4426950408889634f;
 
-enum : int { BSITE_RES = 21, BSITE_X_EMPTY, BSITE_Y_EMPTY, BSITE_X_FULL, BSITE_Y_FULL, BSITE_S_FULL, BSITE_P_FULL,
+__host__ __device__ constexpr uint32_t s_col(int b) { return 64u * static_cast<uint32_t>(b); }
+__host__ __device__ constexpr uint32_t dp_col(int b) { return 128u + 64u * static_cast<uint32_t>(b); }
+
+enum : int { BSITE_RES = 21, BSITE_X_EMPTY, BSITE_Y_EMPTY, BSITE_X_FULL, BSITE_Y_FULL, BSITE_S_FULL, BSITE_DS_FULL,
              BSITE_ACC, BSITE_FINAL };
 
 template <int D>
 struct BLayout {
     static constexpr int CHUNKS = D / 64;
-    static constexpr int CHUNK_BYTES = TILE * 128;
-    static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;
-    static constexpr int STAGES = 2;
+    static constexpr int R_CHUNK_BYTES = TILE * 128;              // 128 rows x 128 bytes
+    static constexpr int R_BYTES = CHUNKS * R_CHUNK_BYTES;        // a resident 128 x d tile
+    static constexpr int H_CHUNK_BYTES = HALF * 128;              // 64 rows x 128 bytes
+    static constexpr int H_BYTES = CHUNKS * H_CHUNK_BYTES;        // a 64 x d half of a walked tile
+    static constexpr int XS = D == 64 ? 6 : 4;                    // ring of K halves (dQ) or Q halves (dK dV)
+    static constexpr int YS = D == 64 ? 6 : 3;                    // ring of V halves or dO halves
     static constexpr int R0_OFF = 0;                              // resident: Q (dQ pass) or K (dK/dV pass)
-    static constexpr int R1_OFF = R0_OFF + TILE_BYTES;            // resident: dO or V
-    static constexpr int X_OFF = R1_OFF + TILE_BYTES;             // ring: K_j or Q_i
-    static constexpr int Y_OFF = X_OFF + STAGES * TILE_BYTES;     // ring: V_j or dO_i
-    static constexpr int BAR_OFF = Y_OFF + STAGES * TILE_BYTES;
-    static constexpr int STAT_OFF = BAR_OFF + 256;                // [2 buffers][L2, D][128] floats
-    static constexpr int SMEM_NEEDED = STAT_OFF + 2 * 2 * TILE * 4 + 1024;
+    static constexpr int R1_OFF = R0_OFF + R_BYTES;               // resident: dO or V
+    static constexpr int X_OFF = R1_OFF + R_BYTES;
+    static constexpr int Y_OFF = X_OFF + XS * H_BYTES;
+    static constexpr int BAR_OFF = Y_OFF + YS * H_BYTES;
+    static constexpr int STAT_OFF = BAR_OFF + 512;                // [2 buffers][L2, D][64] floats
+    static constexpr int SMEM_NEEDED = STAT_OFF + 2 * 2 * HALF * 4 + 1024;
+    // at least 120 KB so that one CTA holds an SM (it allocates all 512 TMEM columns)
     static constexpr int SMEM_BYTES = SMEM_NEEDED > 120 * 1024 ? SMEM_NEEDED : 120 * 1024;
 };
 
-enum : int {
-    BB_RES_FULL = 0,
-    BB_X_FULL = 1,   // + stage
-    BB_X_EMPTY = 3,  // + stage
-    BB_Y_FULL = 5,   // + stage
-    BB_Y_EMPTY = 7,  // + stage
-    BB_S_FULL = 9,
-    BB_P_FULL = 10,
-    BB_ACC_DONE = 11,  // the gradient MMAs of a step have read the dS / P operands in TMEM
-    BB_FINAL = 12,
-    BB_COUNT = 13
+template <int XS, int YS>
+struct BBars {
+    static constexpr int RES_FULL = 0;
+    static constexpr int X_FULL = 1;
+    static constexpr int X_EMPTY = X_FULL + XS;
+    static constexpr int Y_FULL = X_EMPTY + XS;
+    static constexpr int Y_EMPTY = Y_FULL + YS;
+    static constexpr int S_FULL = Y_EMPTY + YS;  // + buffer
+    static constexpr int DS_FULL = S_FULL + 2;   // + buffer
+    static constexpr int ACC_DONE = DS_FULL + 2; // + buffer: the gradient MMAs of a step have read its buffer
+    static constexpr int FINAL = ACC_DONE + 2;
+    static constexpr int COUNT = FINAL + 1;
 };
 
 struct BwdParams {
@@ -106,6 +119,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY, const BwdParams p)
 {
     using L = BLayout<D>;
+    using BB = BBars<L::XS, L::YS>;
+    static_assert(BB::COUNT * 8 + 8 <= 512, "barrier area");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_addr(smem_raw);
     const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
@@ -113,8 +128,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const uint32_t sR0 = sbase + L::R0_OFF, sR1 = sbase + L::R1_OFF, sX = sbase + L::X_OFF, sY = sbase + L::Y_OFF;
     const uint32_t bars = sbase + L::BAR_OFF;
     auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::BAR_OFF + 8 * BB_COUNT);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::BAR_OFF + 8 * BB_COUNT + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::BAR_OFF + 8 * BB::COUNT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::BAR_OFF + 8 * BB::COUNT + 4);
     float* stat = reinterpret_cast<float*>(smem + L::STAT_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -125,8 +140,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 
     if (threadIdx.x == 0) {
         *abort_flag = *reinterpret_cast<volatile int*>(p.err) != 0 ? 1 : 0;
-        for (int i = 0; i < BB_COUNT; ++i)
-            mbar_init(bar(i), i == BB_P_FULL ? 128u : 1u);
+        for (int i = 0; i < BB::COUNT; ++i)
+            mbar_init(bar(i), (i == BB::DS_FULL || i == BB::DS_FULL + 1) ? 128u : 1u);
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -141,93 +156,112 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const bool skip = *abort_flag != 0;
     const int start = p.ptr[tb];
     const int len = skip ? 0 : p.ptr[tb + 1] - start;
+    const int G = 2 * len;  // steps: two 64-row halves per walked tile
 
     if (warp == 4) {
         // ------------------------------------------------------------ producer
-        if (lane == 0 && len > 0) {
-            mbar_arrive_expect_tx(bar(BB_RES_FULL), 2 * L::TILE_BYTES);
+        if (lane == 0 && G > 0) {
+            mbar_arrive_expect_tx(bar(BB::RES_FULL), 2 * L::R_BYTES);
             for (int c = 0; c < L::CHUNKS; ++c) {
-                tma_load_3d(sR0 + c * L::CHUNK_BYTES, &tmR0, bar(BB_RES_FULL), c * 64, tb * TILE, bh);
-                tma_load_3d(sR1 + c * L::CHUNK_BYTES, &tmR1, bar(BB_RES_FULL), c * 64, tb * TILE, bh);
+                tma_load_3d(sR0 + c * L::R_CHUNK_BYTES, &tmR0, bar(BB::RES_FULL), c * 64, tb * TILE, bh);
+                tma_load_3d(sR1 + c * L::R_CHUNK_BYTES, &tmR1, bar(BB::RES_FULL), c * 64, tb * TILE, bh);
             }
             int x_issued = 0, y_issued = 0;
-            for (int j = 0; j < len; ++j) {
-                const int other = p.idx[start + j];
-                const int st = j % L::STAGES;
-                if (j >= L::STAGES && !mbar_wait(bar(BB_X_EMPTY + st), ((j / L::STAGES) - 1) & 1, wc, BSITE_X_EMPTY))
+            for (int g = 0; g < G; ++g) {
+                const int row0 = p.idx[start + (g >> 1)] * TILE + (g & 1) * HALF;
+                const int xs = g % L::XS, ys = g % L::YS;
+                if (g >= L::XS && !mbar_wait(bar(BB::X_EMPTY + xs), ((g / L::XS) - 1) & 1, wc, BSITE_X_EMPTY))
                     break;
-                mbar_arrive_expect_tx(bar(BB_X_FULL + st), L::TILE_BYTES);
+                mbar_arrive_expect_tx(bar(BB::X_FULL + xs), L::H_BYTES);
                 for (int c = 0; c < L::CHUNKS; ++c)
-                    tma_load_3d(sX + st * L::TILE_BYTES + c * L::CHUNK_BYTES, &tmX, bar(BB_X_FULL + st), c * 64,
-                                other * TILE, bh);
-                x_issued = j + 1;
-                if (j >= L::STAGES && !mbar_wait(bar(BB_Y_EMPTY + st), ((j / L::STAGES) - 1) & 1, wc, BSITE_Y_EMPTY))
+                    tma_load_3d(sX + xs * L::H_BYTES + c * L::H_CHUNK_BYTES, &tmX, bar(BB::X_FULL + xs), c * 64,
+                                row0, bh);
+                x_issued = g + 1;
+                if (g >= L::YS && !mbar_wait(bar(BB::Y_EMPTY + ys), ((g / L::YS) - 1) & 1, wc, BSITE_Y_EMPTY))
                     break;
-                mbar_arrive_expect_tx(bar(BB_Y_FULL + st), L::TILE_BYTES);
+                mbar_arrive_expect_tx(bar(BB::Y_FULL + ys), L::H_BYTES);
                 for (int c = 0; c < L::CHUNKS; ++c)
-                    tma_load_3d(sY + st * L::TILE_BYTES + c * L::CHUNK_BYTES, &tmY, bar(BB_Y_FULL + st), c * 64,
-                                other * TILE, bh);
-                y_issued = j + 1;
+                    tma_load_3d(sY + ys * L::H_BYTES + c * L::H_CHUNK_BYTES, &tmY, bar(BB::Y_FULL + ys), c * 64,
+                                row0, bh);
+                y_issued = g + 1;
             }
-            drain_wait(bar(BB_RES_FULL), 0, p.timeout_ns);
-            for (int j = max(0, x_issued - L::STAGES); j < x_issued; ++j)
-                drain_wait(bar(BB_X_FULL + j % L::STAGES), (j / L::STAGES) & 1, p.timeout_ns);
-            for (int j = max(0, y_issued - L::STAGES); j < y_issued; ++j)
-                drain_wait(bar(BB_Y_FULL + j % L::STAGES), (j / L::STAGES) & 1, p.timeout_ns);
+            drain_wait(bar(BB::RES_FULL), 0, p.timeout_ns);
+            for (int g = max(0, x_issued - L::XS); g < x_issued; ++g)
+                drain_wait(bar(BB::X_FULL + g % L::XS), (g / L::XS) & 1, p.timeout_ns);
+            for (int g = max(0, y_issued - L::YS); g < y_issued; ++g)
+                drain_wait(bar(BB::Y_FULL + g % L::YS), (g / L::YS) & 1, p.timeout_ns);
         }
     } else if (warp == 5) {
         // ----------------------------------------------------------------- MMA
-        if (lane == 0 && len > 0) {
-            constexpr uint32_t idesc_nt = idesc_bf16_f32(TILE, TILE, 0, 0);  // A, B K-major
-            constexpr uint32_t idesc_acc = idesc_bf16_f32(TILE, D, 0, 1);    // A from TMEM, B MN-major
-            // D[col] = A(smem tile a) * B(smem tile b)^T over d.
-            auto mma_nt = [&](uint32_t col, uint32_t a, uint32_t b2) {
+        if (lane == 0 && G > 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, HALF, 0, 0);  // A, B K-major, N = 64
+            constexpr uint32_t idesc_acc = idesc_bf16_f32(TILE, D, 0, 1);   // A from TMEM, B MN-major
+            // D[col] = A(resident 128 x d) * B(64-row half)^T over d.
+            auto mma_s = [&](uint32_t col, uint32_t a, uint32_t b2) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
-                    mma_ss(tmem + col, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b2 + off, 16, 1024),
-                           idesc_nt, kk > 0 ? 1u : 0u);
-                }
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + col,
+                           smem_desc_sw128(a + (kk >> 2) * L::R_CHUNK_BYTES + (kk & 3) * 32, 16, 1024),
+                           smem_desc_sw128(b2 + (kk >> 2) * L::H_CHUNK_BYTES + (kk & 3) * 32, 16, 1024), idesc_s,
+                           kk > 0 ? 1u : 0u);
             };
-            // acc[col] += A(TMEM, 128 x 128 bf16 at acol) * B(smem tile b, 128 x d, MN-major).
+            // acc[col] += A(TMEM, 128 x 64 bf16 packed at acol) * B(64-row half, MN-major).
             auto mma_acc = [&](uint32_t col, uint32_t acol, uint32_t b2, bool first) {
 #pragma unroll
-                for (int kk = 0; kk < TILE / 16; ++kk)
-                    mma_ts(tmem + col, tmem + acol + kk * 8, smem_desc_sw128(b2 + kk * 2048, L::CHUNK_BYTES, 1024),
+                for (int kk = 0; kk < HALF / 16; ++kk)
+                    mma_ts(tmem + col, tmem + acol + kk * 8, smem_desc_sw128(b2 + kk * 2048, L::H_CHUNK_BYTES, 1024),
                            idesc_acc, (!first || kk > 0) ? 1u : 0u);
             };
-            bool ok = mbar_wait(bar(BB_RES_FULL), 0, wc, BSITE_RES);
-            tc_fence_after();
-            for (int j = 0; ok && j < len; ++j) {
-                const int st = j % L::STAGES;
-                if (!(ok = mbar_wait(bar(BB_X_FULL + st), (j / L::STAGES) & 1, wc, BSITE_X_FULL)) ||
-                    !(ok = mbar_wait(bar(BB_Y_FULL + st), (j / L::STAGES) & 1, wc, BSITE_Y_FULL)))
-                    break;
-                // The next S / dP overwrite the TMEM columns that the previous
-                // step's gradient MMAs read as operands; MMAs into different
-                // accumulators are not ordered, so wait for those first.
-                if (j > 0 && !(ok = mbar_wait(bar(BB_ACC_DONE), (j - 1) & 1, wc, BSITE_ACC)))
-                    break;
-                tc_fence_after();
-                const uint32_t x = sX + st * L::TILE_BYTES, y = sY + st * L::TILE_BYTES;
-                mma_nt(COL_S, sR0, x);   // S = Q K^T, or S^T = K Q^T
-                mma_nt(COL_DP, sR1, y);  // dP = dO V^T, or dP^T = V dO^T
-                mma_commit(bar(BB_S_FULL));
-                if (!(ok = mbar_wait(bar(BB_P_FULL), j & 1, wc, BSITE_P_FULL)))
-                    break;
-                tc_fence_after();
+            // gradient MMAs of step g (its dS / P in buffer g & 1), then release what it read
+            auto issue_acc = [&](int g) {
+                const int bf = g & 1, xs = g % L::XS, ys = g % L::YS;
+                const uint32_t x = sX + xs * L::H_BYTES, y = sY + ys * L::H_BYTES;
                 if (!TRANS) {
-                    mma_acc(COL_ACC0, COL_S, x, j == 0);   // dQ += dS K
+                    mma_acc(COL_ACC0, s_col(bf), x, g == 0);   // dQ += dS K
                 } else {
-                    mma_acc(COL_ACC1, COL_S, y, j == 0);   // dV += P^T dO
-                    mma_acc(COL_ACC0, COL_DP, x, j == 0);  // dK += dS^T Q
+                    mma_acc(COL_ACC1, s_col(bf), y, g == 0);   // dV += P^T dO
+                    mma_acc(COL_ACC0, dp_col(bf), x, g == 0);  // dK += dS^T Q
                 }
-                mma_commit(bar(BB_ACC_DONE));
-                mma_commit(bar(BB_X_EMPTY + st));
-                mma_commit(bar(BB_Y_EMPTY + st));
+                mma_commit(bar(BB::ACC_DONE + bf));
+                mma_commit(bar(BB::X_EMPTY + xs));
+                if (TRANS)
+                    mma_commit(bar(BB::Y_EMPTY + ys));
+            };
+            bool ok = mbar_wait(bar(BB::RES_FULL), 0, wc, BSITE_RES);
+            tc_fence_after();
+            int acc_issued = 0;
+            for (int g = 0; ok && g < G; ++g) {
+                const int bf = g & 1, xs = g % L::XS, ys = g % L::YS;
+                if (!(ok = mbar_wait(bar(BB::X_FULL + xs), (g / L::XS) & 1, wc, BSITE_X_FULL)) ||
+                    !(ok = mbar_wait(bar(BB::Y_FULL + ys), (g / L::YS) & 1, wc, BSITE_Y_FULL)))
+                    break;
+                // S and dP of this step overwrite buffer bf, which the gradient
+                // MMAs of step g - 2 read; MMAs into different accumulators are
+                // not ordered, so wait for those first.
+                if (g >= 2 && !(ok = mbar_wait(bar(BB::ACC_DONE + bf), ((g - 2) >> 1) & 1, wc, BSITE_ACC)))
+                    break;
+                tc_fence_after();
+                mma_s(s_col(bf), sR0, sX + xs * L::H_BYTES);   // S = Q K^T, or S^T = K Q^T
+                mma_s(dp_col(bf), sR1, sY + ys * L::H_BYTES);  // dP = dO V^T, or dP^T = V dO^T
+                mma_commit(bar(BB::S_FULL + bf));
+                if (!TRANS)
+                    mma_commit(bar(BB::Y_EMPTY + ys));  // V half no longer needed
+                if (g >= 1) {
+                    if (!(ok = mbar_wait(bar(BB::DS_FULL + (bf ^ 1)), ((g - 1) >> 1) & 1, wc, BSITE_DS_FULL)))
+                        break;
+                    tc_fence_after();
+                    issue_acc(g - 1);
+                    acc_issued = g;
+                }
             }
-            mma_commit(bar(BB_FINAL));
-            drain_wait(bar(BB_FINAL), 0, p.timeout_ns);
+            if (ok && acc_issued == G - 1) {
+                if (mbar_wait(bar(BB::DS_FULL + ((G - 1) & 1)), ((G - 1) >> 1) & 1, wc, BSITE_DS_FULL)) {
+                    tc_fence_after();
+                    issue_acc(G - 1);
+                }
+            }
+            mma_commit(bar(BB::FINAL));
+            drain_wait(bar(BB::FINAL), 0, p.timeout_ns);
         }
     } else {
         // ------------------------------------------------------ gradient warps
@@ -241,48 +275,56 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         const float row_l2 = (!TRANS && row_valid) ? p.lse[static_cast<size_t>(bh) * n + row] * LOG2E : 0.f;
         const float row_d = (!TRANS && row_valid) ? p.Dv[static_cast<size_t>(bh) * n + row] : 0.f;
         bool ok = true;
-        for (int j = 0; j < len; ++j) {
+        uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
+        bool masked = false;
+        for (int g = 0; g < G; ++g) {
+            const int j = g >> 1, half = g & 1, bf = g & 1;
             const int other = p.idx[start + j];  // key tile (dQ) or query tile (dK/dV)
-            const bool partial = p.flag[start + j] != RA_TILE_FULL;
-            float* st_l2 = stat + (j & 1) * 2 * TILE;
-            float* st_d = st_l2 + TILE;
+            float* st_l2 = stat + bf * 2 * HALF;
+            float* st_d = st_l2 + HALF;
             if (TRANS) {
-                // statistics of the query tile's 128 columns; columns >= n get
+                // statistics of the step's 64 query columns; columns >= n get
                 // L = +inf so their P is exactly 0
-                const int q = other * TILE + t;
-                st_l2[t] = q < n ? p.lse[static_cast<size_t>(bh) * n + q] * LOG2E : INFINITY;
-                st_d[t] = q < n ? p.Dv[static_cast<size_t>(bh) * n + q] : 0.f;
+                const int q = other * TILE + half * HALF + (t & (HALF - 1));
+                if (t < HALF)
+                    st_l2[t] = q < n ? p.lse[static_cast<size_t>(bh) * n + q] * LOG2E : INFINITY;
+                else
+                    st_d[t - HALF] = q < n ? p.Dv[static_cast<size_t>(bh) * n + q] : 0.f;
             }
-            uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
-            const bool use_family = p.mode == RA_MODE_TOKEN_EXACT && partial;
-            const bool masked = use_family || (!TRANS && tail && other == p.nb - 1);
-            if (masked) {
-                if (use_family && row_valid) {
-                    if (!TRANS)
-                        row_keep_mask(p.g, rf, rp, other * TILE, mk[0], mk[1], mk[2], mk[3]);
-                    else
-                        col_keep_mask(p.g, rf, rp, other * TILE, mk[0], mk[1], mk[2], mk[3]);
-                } else if (!TRANS) {
-                    const int valid_cols = min(TILE, n - other * TILE);
+            if (half == 0) {
+                const bool partial = p.flag[start + j] != RA_TILE_FULL;
+                const bool use_family = p.mode == RA_MODE_TOKEN_EXACT && partial;
+                masked = use_family || (!TRANS && tail && other == p.nb - 1);
+                mk[0] = mk[1] = mk[2] = mk[3] = ~0u;
+                if (masked) {
+                    if (use_family && row_valid) {
+                        if (!TRANS)
+                            row_keep_mask(p.g, rf, rp, other * TILE, mk[0], mk[1], mk[2], mk[3]);
+                        else
+                            col_keep_mask(p.g, rf, rp, other * TILE, mk[0], mk[1], mk[2], mk[3]);
+                    } else if (!TRANS) {
+                        const int valid_cols = min(TILE, n - other * TILE);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int v = valid_cols - 32 * c;
-                        mk[c] = v >= 32 ? 0xFFFFFFFFu : (v <= 0 ? 0u : ((1u << v) - 1u));
+                        for (int c = 0; c < 4; ++c) {
+                            const int v = valid_cols - 32 * c;
+                            mk[c] = v >= 32 ? 0xFFFFFFFFu : (v <= 0 ? 0u : ((1u << v) - 1u));
+                        }
                     }
                 }
             }
-            ok = mbar_wait(bar(BB_S_FULL), j & 1, wc, BSITE_S_FULL);
+            ok = mbar_wait(bar(BB::S_FULL + bf), (g >> 1) & 1, wc, BSITE_S_FULL);
             // one decision for all 128 threads; also publishes the staged statistics
             ok = TRANS ? sync_and_128(ok) : __all_sync(0xFFFFFFFFu, ok);
             if (!ok)
                 break;
             tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
                 uint32_t sv[32], dv[32];
-                tmem_ld32(lane_base + COL_S + c * 32, sv);
-                tmem_ld32(lane_base + COL_DP + c * 32, dv);
+                tmem_ld32(lane_base + s_col(bf) + c * 32, sv);
+                tmem_ld32(lane_base + dp_col(bf) + c * 32, dv);
                 tmem_wait_ld();
+                const uint32_t mword = half ? (c ? mk[3] : mk[2]) : (c ? mk[1] : mk[0]);
                 uint32_t pk[16], dk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
@@ -290,7 +332,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const int col = c * 32 + e + u;
-                        const bool keep = !masked || ((mk[c] >> (e + u)) & 1u);
+                        const bool keep = !masked || ((mword >> (e + u)) & 1u);
                         const float l2 = TRANS ? st_l2[col] : row_l2;
                         const float dd = TRANS ? st_d[col] : row_d;
                         const float x = fmaf(__uint_as_float(sv[e + u]), p.scale_log2, -l2);
@@ -302,21 +344,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                 }
                 // Written over columns already read (chunk c goes to columns 16 c .. 16 c + 15).
                 if (!TRANS) {
-                    tmem_st16(lane_base + COL_S + c * 16, dk);   // dS for dQ += dS K
+                    tmem_st16(lane_base + s_col(bf) + c * 16, dk);   // dS for dQ += dS K
                 } else {
-                    tmem_st16(lane_base + COL_S + c * 16, pk);   // P^T for dV += P^T dO
-                    tmem_st16(lane_base + COL_DP + c * 16, dk);  // dS^T for dK += dS^T Q
+                    tmem_st16(lane_base + s_col(bf) + c * 16, pk);   // P^T for dV += P^T dO
+                    tmem_st16(lane_base + dp_col(bf) + c * 16, dk);  // dS^T for dK += dS^T Q
                 }
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(BB_P_FULL));
+            mbar_arrive(bar(BB::DS_FULL + bf));
         }
         // ------------------------------------------------------------ epilogue
-        if (len > 0 && ok)
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(BB_FINAL), 0, wc, BSITE_FINAL));
+        if (G > 0 && ok)
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(BB::FINAL), 0, wc, BSITE_FINAL));
         tc_fence_after();
-        if (ok && !*abort_flag && row_valid) {
+        // tcgen05.ld is warp-collective: every lane loads, only rows < n store
+        if (__all_sync(0xFFFFFFFFu, ok && !*abort_flag)) {
 #pragma unroll 1
             for (int which = 0; which < (TRANS ? 2 : 1); ++which) {
                 __nv_bfloat16* dst_row = (which == 0 ? p.out0 : p.out1) + (static_cast<size_t>(bh) * n + row) * D;
@@ -325,7 +368,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
-                    if (len > 0) {
+                    if (G > 0) {
                         tmem_ld32(lane_base + col0 + c * 32, o);
                         tmem_wait_ld();
                     } else {
@@ -338,10 +381,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
                     for (int e = 0; e < 32; e += 2)
                         w[e >> 1] = pack_bf16(__uint_as_float(o[e]) * mul, __uint_as_float(o[e + 1]) * mul);
-                    uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+                    if (row_valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        dst[u] = v[u];
+                        for (int u = 0; u < 4; ++u)
+                            dst[u] = v[u];
+                    }
                 }
             }
         }
@@ -411,9 +456,12 @@ ra_status run_bwd(const void* Q, const void* K, const void* V, const void* O, co
     ra_status st = cuda_fail(cudaGetLastError(), "bwd_dot_kernel launch");
     if (st != RA_OK)
         return st;
-    CUtensorMap mq, mk, mv, mdo;
-    if ((st = make_map(&mq, Q, BH, n, D, TILE)) != RA_OK || (st = make_map(&mk, K, BH, n, D, TILE)) != RA_OK ||
-        (st = make_map(&mv, V, BH, n, D, TILE)) != RA_OK || (st = make_map(&mdo, dO, BH, n, D, TILE)) != RA_OK)
+    // resident tiles: 128-row boxes; walked tiles: 64-row halves
+    CUtensorMap rq, rk, rv, rdo, hq, hk, hv, hdo;
+    if ((st = make_map(&rq, Q, BH, n, D, TILE)) != RA_OK || (st = make_map(&rdo, dO, BH, n, D, TILE)) != RA_OK ||
+        (st = make_map(&rk, K, BH, n, D, TILE)) != RA_OK || (st = make_map(&rv, V, BH, n, D, TILE)) != RA_OK ||
+        (st = make_map(&hq, Q, BH, n, D, HALF)) != RA_OK || (st = make_map(&hdo, dO, BH, n, D, HALF)) != RA_OK ||
+        (st = make_map(&hk, K, BH, n, D, HALF)) != RA_OK || (st = make_map(&hv, V, BH, n, D, HALF)) != RA_OK)
         return st;
     BwdParams p;
     std::memset(&p, 0, sizeof p);
@@ -428,21 +476,21 @@ ra_status run_bwd(const void* Q, const void* K, const void* V, const void* O, co
     p.timeout_ns = wait_timeout_ns();
     if ((st = device_error_word(&p.err)) != RA_OK)
         return st;
-    // dQ: query tiles over the block-CSR rows; resident Q, dO; ring K, V
+    // dQ: query tiles over the block-CSR rows; resident Q, dO; rings of K, V halves
     p.ptr = m->row_ptr;
     p.idx = m->col_idx;
     p.flag = m->flag;
     p.out0 = static_cast<__nv_bfloat16*>(dQ);
     p.out1 = nullptr;
-    if ((st = launch_bwd<D, false>(mq, mdo, mk, mv, p, B, cs)) != RA_OK)
+    if ((st = launch_bwd<D, false>(rq, rdo, hk, hv, p, B, cs)) != RA_OK)
         return st;
-    // dK, dV: key tiles over the transposed block-CSR; resident K, V; ring Q, dO
+    // dK, dV: key tiles over the transposed block-CSR; resident K, V; rings of Q, dO halves
     p.ptr = m->col_ptr;
     p.idx = m->row_idx;
     p.flag = m->tflag;
     p.out0 = static_cast<__nv_bfloat16*>(dK);
     p.out1 = static_cast<__nv_bfloat16*>(dV);
-    return launch_bwd<D, true>(mk, mv, mq, mdo, p, B, cs);
+    return launch_bwd<D, true>(rk, rv, hq, hdo, p, B, cs);
 }
 
 }  // namespace
@@ -454,7 +502,7 @@ extern "C" ra_status ra_attention_bwd(const void* Q, const void* K, const void* 
                                       const float* lse, void* dQ, void* dK, void* dV, float* D_workspace, int B,
                                       int H, int d, const ra_mask* m, float scale, int mode, ra_stream stream)
 {
-    const void* ptrs[9] = {Q, K, V, O, dO, dQ, dK, dV, nullptr};
+    const void* ptrs[8] = {Q, K, V, O, dO, dQ, dK, dV};
     for (int i = 0; i < 8; ++i) {
         if (!ptrs[i])
             return fail(RA_ERR_INVALID_ARG, "NULL tensor pointer");
