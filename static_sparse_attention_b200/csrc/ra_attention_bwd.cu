@@ -401,6 +401,308 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// dQ kernel with 128-key steps.  A tcgen05.mma of M = 128 runs at the full
+// rate only for N >= 128 (N = 64 reaches about two thirds), so S = Q K^T and
+// dP = dO V^T are computed for a whole 128-key tile per step.  TMEM: S in two
+// buffers (columns 0 and 128), dP in one (256; the gradient warps load it into
+// registers first and release it at once), dQ at 384.  The MMA warp issues
+// dP_j, then S_j, then the gradient MMA of step j - 1, so that its wait for the
+// gradient MMA of step j - 2 (whose dS buffer S_j overwrites) overlaps dP_j.
+// 320 threads: two gradient warpgroups (columns 64 wg .. 64 wg + 63 of each
+// step), warp 8 issues the TMA loads, warp 9 the MMAs.
+constexpr int DQ_THREADS = 320, DQ_GRAD_THREADS = 256, DQ_PRODUCER_WARP = 8, DQ_MMA_WARP = 9;
+constexpr uint32_t DQ_COL_DP = 256, DQ_COL_ACC = 384;
+__host__ __device__ constexpr uint32_t dq_s_col(int b) { return 128u * static_cast<uint32_t>(b); }
+
+template <int D>
+struct DqLayout {
+    static constexpr int CHUNKS = D / 64;
+    static constexpr int CHUNK_BYTES = TILE * 128;          // 128 rows x 128 bytes
+    static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES; // a 128 x d tile
+    static constexpr int KS = D == 64 ? 3 : 2;               // K tile ring
+    static constexpr int VS = D == 64 ? 3 : 2;               // V tile ring
+    static constexpr int Q_OFF = 0, DO_OFF = TILE_BYTES;
+    static constexpr int K_OFF = 2 * TILE_BYTES;
+    static constexpr int V_OFF = K_OFF + KS * TILE_BYTES;
+    static constexpr int BAR_OFF = V_OFF + VS * TILE_BYTES;
+    static constexpr int SMEM_NEEDED = BAR_OFF + 256 + 1024;
+    static constexpr int SMEM_BYTES = SMEM_NEEDED > 120 * 1024 ? SMEM_NEEDED : 120 * 1024;
+};
+
+template <int KS, int VS>
+struct DqBars {
+    static constexpr int RES_FULL = 0;
+    static constexpr int K_FULL = 1;
+    static constexpr int K_EMPTY = K_FULL + KS;
+    static constexpr int V_FULL = K_EMPTY + KS;
+    static constexpr int V_EMPTY = V_FULL + VS;
+    static constexpr int S_FULL = V_EMPTY + VS;  // + buffer: S_j and dP_j complete
+    static constexpr int DP_FREE = S_FULL + 2;   // the gradient warps have loaded dP
+    static constexpr int DS_FULL = DP_FREE + 1;  // + buffer: dS of the step written
+    static constexpr int ACC_DONE = DS_FULL + 2; // + buffer: dQ += dS K of the step complete
+    static constexpr int FINAL = ACC_DONE + 2;
+    static constexpr int COUNT = FINAL + 1;
+};
+
+template <int D>
+__global__ void __launch_bounds__(DQ_THREADS, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const BwdParams p)
+{
+    using L = DqLayout<D>;
+    using BB = DqBars<L::KS, L::VS>;
+    static_assert(BB::COUNT * 8 + 8 <= 256, "barrier area");
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_addr(smem_raw);
+    const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (sbase - raw_addr);
+    const uint32_t sQ = sbase + L::Q_OFF, sDO = sbase + L::DO_OFF, sK = sbase + L::K_OFF, sV = sbase + L::V_OFF;
+    const uint32_t bars = sbase + L::BAR_OFF;
+    auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::BAR_OFF + 8 * BB::COUNT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::BAR_OFF + 8 * BB::COUNT + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int bh = b * p.H + h;
+    const int n = p.g.n;
+    WaitCtl wc{abort_flag, p.err, p.timeout_ns};
+
+    if (threadIdx.x == 0) {
+        *abort_flag = *reinterpret_cast<volatile int*>(p.err) != 0 ? 1 : 0;
+        for (int i = 0; i < BB::COUNT; ++i) {
+            const bool grad = i == BB::DP_FREE || i == BB::DS_FULL || i == BB::DS_FULL + 1;
+            mbar_init(bar(i), grad ? static_cast<uint32_t>(DQ_GRAD_THREADS) : 1u);
+        }
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == DQ_MMA_WARP) {
+        tmem_alloc(smem_addr(tmem_slot), BWD_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const bool skip = *abort_flag != 0;
+    const int start = p.ptr[qb];
+    const int len = skip ? 0 : p.ptr[qb + 1] - start;
+
+    if (warp == DQ_PRODUCER_WARP) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0 && len > 0) {
+            mbar_arrive_expect_tx(bar(BB::RES_FULL), 2 * L::TILE_BYTES);
+            for (int c = 0; c < L::CHUNKS; ++c) {
+                tma_load_3d(sQ + c * L::CHUNK_BYTES, &tmQ, bar(BB::RES_FULL), c * 64, qb * TILE, bh);
+                tma_load_3d(sDO + c * L::CHUNK_BYTES, &tmDO, bar(BB::RES_FULL), c * 64, qb * TILE, bh);
+            }
+            int k_issued = 0, v_issued = 0;
+            for (int j = 0; j < len; ++j) {
+                const int row0 = p.idx[start + j] * TILE;
+                const int ks = j % L::KS, vs = j % L::VS;
+                if (j >= L::VS && !mbar_wait(bar(BB::V_EMPTY + vs), ((j / L::VS) - 1) & 1, wc, BSITE_Y_EMPTY))
+                    break;
+                mbar_arrive_expect_tx(bar(BB::V_FULL + vs), L::TILE_BYTES);
+                for (int c = 0; c < L::CHUNKS; ++c)
+                    tma_load_3d(sV + vs * L::TILE_BYTES + c * L::CHUNK_BYTES, &tmV, bar(BB::V_FULL + vs), c * 64, row0,
+                                bh);
+                v_issued = j + 1;
+                if (j >= L::KS && !mbar_wait(bar(BB::K_EMPTY + ks), ((j / L::KS) - 1) & 1, wc, BSITE_X_EMPTY))
+                    break;
+                mbar_arrive_expect_tx(bar(BB::K_FULL + ks), L::TILE_BYTES);
+                for (int c = 0; c < L::CHUNKS; ++c)
+                    tma_load_3d(sK + ks * L::TILE_BYTES + c * L::CHUNK_BYTES, &tmK, bar(BB::K_FULL + ks), c * 64, row0,
+                                bh);
+                k_issued = j + 1;
+            }
+            drain_wait(bar(BB::RES_FULL), 0, p.timeout_ns);
+            for (int j = max(0, k_issued - L::KS); j < k_issued; ++j)
+                drain_wait(bar(BB::K_FULL + j % L::KS), (j / L::KS) & 1, p.timeout_ns);
+            for (int j = max(0, v_issued - L::VS); j < v_issued; ++j)
+                drain_wait(bar(BB::V_FULL + j % L::VS), (j / L::VS) & 1, p.timeout_ns);
+        }
+    } else if (warp == DQ_MMA_WARP) {
+        // ----------------------------------------------------------------- MMA
+        if (lane == 0 && len > 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, TILE, 0, 0);  // A, B K-major, N = 128
+            constexpr uint32_t idesc_acc = idesc_bf16_f32(TILE, D, 0, 1);   // A from TMEM, B MN-major
+            // D[col] = A(resident 128 x d) * B(128-row tile)^T over d.
+            auto mma_s = [&](uint32_t col, uint32_t a, uint32_t b2) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
+                    mma_ss(tmem + col, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b2 + off, 16, 1024),
+                           idesc_s, kk > 0 ? 1u : 0u);
+                }
+            };
+            // dQ += dS_j K_j: dS packed by the warpgroups, keys 16 kk .. 16 kk + 15
+            // at columns 64 (kk / 4) + 8 (kk % 4) of the step's S buffer.
+            auto issue_acc = [&](int j) {
+                const int bf = j & 1, ks = j % L::KS;
+                const uint32_t kbase = sK + ks * L::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < TILE / 16; ++kk)
+                    mma_ts(tmem + DQ_COL_ACC, tmem + dq_s_col(bf) + (kk >> 2) * 64 + (kk & 3) * 8,
+                           smem_desc_sw128(kbase + kk * 2048, L::CHUNK_BYTES, 1024), idesc_acc,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar(BB::ACC_DONE + bf));
+                mma_commit(bar(BB::K_EMPTY + ks));
+            };
+            bool ok = mbar_wait(bar(BB::RES_FULL), 0, wc, BSITE_RES);
+            tc_fence_after();
+            int acc_issued = 0;
+            for (int j = 0; ok && j < len; ++j) {
+                const int bf = j & 1, ks = j % L::KS, vs = j % L::VS;
+                // dP_j into the single dP buffer, once the gradient warps have loaded dP_{j-1}
+                if (!(ok = mbar_wait(bar(BB::V_FULL + vs), (j / L::VS) & 1, wc, BSITE_Y_FULL)))
+                    break;
+                if (j >= 1 && !(ok = mbar_wait(bar(BB::DP_FREE), (j - 1) & 1, wc, BSITE_DS_FULL)))
+                    break;
+                tc_fence_after();
+                mma_s(DQ_COL_DP, sDO, sV + vs * L::TILE_BYTES);
+                mma_commit(bar(BB::V_EMPTY + vs));
+                // S_j into buffer bf, once the gradient MMA of step j - 2 (which read
+                // dS from that buffer) has completed: MMAs into different
+                // accumulators are not ordered
+                if (!(ok = mbar_wait(bar(BB::K_FULL + ks), (j / L::KS) & 1, wc, BSITE_X_FULL)))
+                    break;
+                if (j >= 2 && !(ok = mbar_wait(bar(BB::ACC_DONE + bf), ((j - 2) >> 1) & 1, wc, BSITE_ACC)))
+                    break;
+                tc_fence_after();
+                mma_s(dq_s_col(bf), sQ, sK + ks * L::TILE_BYTES);
+                mma_commit(bar(BB::S_FULL + bf));
+                if (j >= 1) {
+                    if (!(ok = mbar_wait(bar(BB::DS_FULL + (bf ^ 1)), ((j - 1) >> 1) & 1, wc, BSITE_DS_FULL)))
+                        break;
+                    tc_fence_after();
+                    issue_acc(j - 1);
+                    acc_issued = j;
+                }
+            }
+            if (ok && acc_issued == len - 1) {
+                if (mbar_wait(bar(BB::DS_FULL + ((len - 1) & 1)), ((len - 1) >> 1) & 1, wc, BSITE_DS_FULL)) {
+                    tc_fence_after();
+                    issue_acc(len - 1);
+                }
+            }
+            mma_commit(bar(BB::FINAL));
+            drain_wait(bar(BB::FINAL), 0, p.timeout_ns);
+        }
+    } else {
+        // ------------------------------------------------------ gradient warps
+        const int wg = warp >> 2;            // warpgroup: columns 64 wg .. 64 wg + 63 of each step
+        const int t = threadIdx.x & 127;     // == TMEM lane: query row of the tile
+        const int row = qb * TILE + t;
+        const bool row_valid = row < n;
+        const int rf = row_valid ? row / p.g.s : 0, rp = row_valid ? row % p.g.s : 0;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const uint32_t my_col = 64u * static_cast<uint32_t>(wg);
+        const bool tail = (n % TILE) != 0;
+        const float row_l2 = row_valid ? p.lse[static_cast<size_t>(bh) * n + row] * LOG2E : 0.f;
+        const float row_d = row_valid ? p.Dv[static_cast<size_t>(bh) * n + row] : 0.f;
+        bool ok = true;
+        for (int j = 0; j < len; ++j) {
+            const int bf = j & 1;
+            const int kb = p.idx[start + j];
+            const bool use_family = p.mode == RA_MODE_TOKEN_EXACT && p.flag[start + j] != RA_TILE_FULL;
+            const bool masked = use_family || (tail && kb == p.nb - 1);
+            uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
+            if (masked) {
+                if (use_family && row_valid) {
+                    row_keep_mask(p.g, rf, rp, kb * TILE, mk[0], mk[1], mk[2], mk[3]);
+                } else {
+                    const int valid_cols = min(TILE, n - kb * TILE);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int v = valid_cols - 32 * c;
+                        mk[c] = v >= 32 ? 0xFFFFFFFFu : (v <= 0 ? 0u : ((1u << v) - 1u));
+                    }
+                }
+            }
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(BB::S_FULL + bf), (j >> 1) & 1, wc, BSITE_S_FULL));
+            if (!ok)
+                break;
+            tc_fence_after();
+            // dP first, then release the dP buffer for the next step's MMA
+            uint32_t dv[2][32];
+            tmem_ld32(lane_base + DQ_COL_DP + my_col, dv[0]);
+            tmem_ld32(lane_base + DQ_COL_DP + my_col + 32, dv[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar(BB::DP_FREE));
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t sv[32];
+                tmem_ld32(lane_base + dq_s_col(bf) + my_col + c * 32, sv);
+                tmem_wait_ld();
+                const uint32_t mword = wg ? (c ? mk[3] : mk[2]) : (c ? mk[1] : mk[0]);
+                uint32_t dk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float ds[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const bool keep = !masked || ((mword >> (e + u)) & 1u);
+                        const float x = fmaf(__uint_as_float(sv[e + u]), p.scale_log2, -row_l2);
+                        const float pe = keep ? fast_exp2(x) : 0.f;
+                        ds[u] = pe * (__uint_as_float(dv[c][e + u]) - row_d);
+                    }
+                    dk[e >> 1] = pack_bf16(ds[0], ds[1]);
+                }
+                // Packed into columns this warpgroup has already read.
+                tmem_st16(lane_base + dq_s_col(bf) + my_col + c * 16, dk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(BB::DS_FULL + bf));
+        }
+        // ------------------------------------------------------------ epilogue
+        if (len > 0 && ok)
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(BB::FINAL), 0, wc, BSITE_FINAL));
+        tc_fence_after();
+        // tcgen05.ld is warp-collective: every lane loads, only rows < n store;
+        // warpgroup wg stores dQ columns [wg d/2, (wg + 1) d/2)
+        if (__all_sync(0xFFFFFFFFu, ok && !*abort_flag)) {
+            __nv_bfloat16* dst_row = p.out0 + (static_cast<size_t>(bh) * n + row) * D;
+            constexpr int C_PER_WG = D / 64;
+#pragma unroll
+            for (int cc = 0; cc < C_PER_WG; ++cc) {
+                const int c = wg * C_PER_WG + cc;
+                uint32_t o[32];
+                if (len > 0) {
+                    tmem_ld32(lane_base + DQ_COL_ACC + c * 32, o);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        o[e] = 0u;
+                }
+                uint4 v[4];
+                uint32_t* w = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+                for (int e = 0; e < 32; e += 2)
+                    w[e >> 1] = pack_bf16(__uint_as_float(o[e]) * p.scale, __uint_as_float(o[e + 1]) * p.scale);
+                if (row_valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        dst[u] = v[u];
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == DQ_MMA_WARP) {
+        __syncwarp();
+        tmem_dealloc(tmem, BWD_TMEM_COLS);
+    }
+}
+
 // D[r] = <dO[r], O[r]> over d, one warp per row.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_dot_kernel(const __nv_bfloat16* __restrict__ O,
@@ -444,6 +746,23 @@ ra_status launch_bwd(const CUtensorMap& r0, const CUtensorMap& r1, const CUtenso
 }
 
 template <int D>
+ra_status launch_dq(const CUtensorMap& q, const CUtensorMap& dO, const CUtensorMap& k, const CUtensorMap& v,
+                    const BwdParams& p, int B, cudaStream_t cs)
+{
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        DqLayout<D>::SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess)
+        return cuda_fail(attr_err, "cudaFuncSetAttribute(bwd_dq_kernel)");
+    dim3 grid(p.nb, p.H, B);
+    bwd_dq_kernel<D><<<grid, DQ_THREADS, DqLayout<D>::SMEM_BYTES, cs>>>(q, dO, k, v, p);
+    return cuda_fail(cudaGetLastError(), "bwd_dq_kernel launch");
+}
+
+template <int D>
 ra_status run_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* lse,
                   void* dQ, void* dK, void* dV, float* Dws, int B, int H, const ra_mask* m, float scale, int mode,
                   cudaStream_t cs)
@@ -457,11 +776,10 @@ ra_status run_bwd(const void* Q, const void* K, const void* V, const void* O, co
     if (st != RA_OK)
         return st;
     // resident tiles: 128-row boxes; walked tiles: 64-row halves
-    CUtensorMap rq, rk, rv, rdo, hq, hk, hv, hdo;
+    CUtensorMap rq, rk, rv, rdo, hq, hdo;
     if ((st = make_map(&rq, Q, BH, n, D, TILE)) != RA_OK || (st = make_map(&rdo, dO, BH, n, D, TILE)) != RA_OK ||
         (st = make_map(&rk, K, BH, n, D, TILE)) != RA_OK || (st = make_map(&rv, V, BH, n, D, TILE)) != RA_OK ||
-        (st = make_map(&hq, Q, BH, n, D, HALF)) != RA_OK || (st = make_map(&hdo, dO, BH, n, D, HALF)) != RA_OK ||
-        (st = make_map(&hk, K, BH, n, D, HALF)) != RA_OK || (st = make_map(&hv, V, BH, n, D, HALF)) != RA_OK)
+        (st = make_map(&hq, Q, BH, n, D, HALF)) != RA_OK || (st = make_map(&hdo, dO, BH, n, D, HALF)) != RA_OK)
         return st;
     BwdParams p;
     std::memset(&p, 0, sizeof p);
@@ -476,13 +794,13 @@ ra_status run_bwd(const void* Q, const void* K, const void* V, const void* O, co
     p.timeout_ns = wait_timeout_ns();
     if ((st = device_error_word(&p.err)) != RA_OK)
         return st;
-    // dQ: query tiles over the block-CSR rows; resident Q, dO; rings of K, V halves
+    // dQ: query tiles over the block-CSR rows; resident Q, dO; rings of whole K, V tiles
     p.ptr = m->row_ptr;
     p.idx = m->col_idx;
     p.flag = m->flag;
     p.out0 = static_cast<__nv_bfloat16*>(dQ);
     p.out1 = nullptr;
-    if ((st = launch_bwd<D, false>(rq, rdo, hk, hv, p, B, cs)) != RA_OK)
+    if ((st = launch_dq<D>(rq, rdo, rk, rv, p, B, cs)) != RA_OK)
         return st;
     // dK, dV: key tiles over the transposed block-CSR; resident K, V; rings of Q, dO halves
     p.ptr = m->col_ptr;
