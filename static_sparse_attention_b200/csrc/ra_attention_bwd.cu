@@ -7,21 +7,18 @@
 //   dQ = scale dS K,   dK = scale dS^T Q,   dV = P^T dO.
 // Deterministic: no atomics, each output tile is owned by one CTA.
 //
-//   bwd_dot_kernel         D = rowsum(dO * O) (fp32), one warp per row.
-//   bwd_kernel<D, false>   one CTA per query tile, walking its block-CSR row:
+//   bwd_dot_kernel     D = rowsum(dO * O) (fp32), one warp per row.
+//   bwd_dq_kernel      one CTA per query tile, walking its block-CSR row:
 //       S = Q K^T and dP = dO V^T (tcgen05.mma into TMEM), dS (registers,
 //       bf16 back into TMEM), dQ += dS K (A = dS from TMEM).
-//   bwd_kernel<D, true>    one CTA per key tile, walking the transposed CSR:
-//       S^T = K Q^T and dP^T = V dO^T, P^T and dS^T (bf16 into TMEM),
-//       dV += P^T dO and dK += dS^T Q.
-// Both recompute P from L instead of storing it.  The walked tiles are taken
-// in 64-row halves ("steps"): the MMAs of step g run while the gradient warps
-// turn step g-1's S and dP into dS, with two TMEM buffers for S and dP.
-// 192 threads: warps 0-3 own one resident row each per thread (TMEM lane =
-// row), warp 4 issues the TMA loads (two resident 128-row tiles, two rings of
-// 64-row halves), warp 5 allocates TMEM and issues the MMAs.
-// TMEM columns: S buffers at 0 and 64, dP buffers at 128 and 192, the
-// accumulators at 256 (dQ or dK) and 384 (dV).
+//   bwd_dkdv_kernel    one CTA per key tile, walking the transposed CSR:
+//       S^T = K Q^T and dP^T = V dO^T, P^T (bf16 into shared memory) and
+//       dS^T (bf16 into TMEM), dK += dS^T Q and dV += P^T dO.
+// Both recompute P from L instead of storing it, and take the walked side one
+// 128-row tile per step, so that every product is an M = 128, N >= 128
+// tcgen05.mma (N = 64 runs at about two thirds of the rate).  Each has 320
+// threads: two gradient warpgroups that split the step's 128 columns (a thread
+// owns one resident row; TMEM lane = row), a TMA producer warp and an MMA warp.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -36,51 +33,11 @@
 namespace ra {
 namespace {
 
-constexpr int BWD_THREADS = 192;
-constexpr int HALF = 64;
 constexpr uint32_t BWD_TMEM_COLS = 512;
-constexpr uint32_t COL_ACC0 = 256, COL_ACC1 = 384;
 constexpr float LOG2E = 1.4426950408889634f;
-
-__host__ __device__ constexpr uint32_t s_col(int b) { return 64u * static_cast<uint32_t>(b); }
-__host__ __device__ constexpr uint32_t dp_col(int b) { return 128u + 64u * static_cast<uint32_t>(b); }
 
 enum : int { BSITE_RES = 21, BSITE_X_EMPTY, BSITE_Y_EMPTY, BSITE_X_FULL, BSITE_Y_FULL, BSITE_S_FULL, BSITE_DS_FULL,
              BSITE_ACC, BSITE_FINAL };
-
-template <int D>
-struct BLayout {
-    static constexpr int CHUNKS = D / 64;
-    static constexpr int R_CHUNK_BYTES = TILE * 128;              // 128 rows x 128 bytes
-    static constexpr int R_BYTES = CHUNKS * R_CHUNK_BYTES;        // a resident 128 x d tile
-    static constexpr int H_CHUNK_BYTES = HALF * 128;              // 64 rows x 128 bytes
-    static constexpr int H_BYTES = CHUNKS * H_CHUNK_BYTES;        // a 64 x d half of a walked tile
-    static constexpr int XS = D == 64 ? 6 : 4;                    // ring of K halves (dQ) or Q halves (dK dV)
-    static constexpr int YS = D == 64 ? 6 : 3;                    // ring of V halves or dO halves
-    static constexpr int R0_OFF = 0;                              // resident: Q (dQ pass) or K (dK/dV pass)
-    static constexpr int R1_OFF = R0_OFF + R_BYTES;               // resident: dO or V
-    static constexpr int X_OFF = R1_OFF + R_BYTES;
-    static constexpr int Y_OFF = X_OFF + XS * H_BYTES;
-    static constexpr int BAR_OFF = Y_OFF + YS * H_BYTES;
-    static constexpr int STAT_OFF = BAR_OFF + 512;                // [2 buffers][L2, D][64] floats
-    static constexpr int SMEM_NEEDED = STAT_OFF + 2 * 2 * HALF * 4 + 1024;
-    // at least 120 KB so that one CTA holds an SM (it allocates all 512 TMEM columns)
-    static constexpr int SMEM_BYTES = SMEM_NEEDED > 120 * 1024 ? SMEM_NEEDED : 120 * 1024;
-};
-
-template <int XS, int YS>
-struct BBars {
-    static constexpr int RES_FULL = 0;
-    static constexpr int X_FULL = 1;
-    static constexpr int X_EMPTY = X_FULL + XS;
-    static constexpr int Y_FULL = X_EMPTY + XS;
-    static constexpr int Y_EMPTY = Y_FULL + YS;
-    static constexpr int S_FULL = Y_EMPTY + YS;  // + buffer
-    static constexpr int DS_FULL = S_FULL + 2;   // + buffer
-    static constexpr int ACC_DONE = DS_FULL + 2; // + buffer: the gradient MMAs of a step have read its buffer
-    static constexpr int FINAL = ACC_DONE + 2;
-    static constexpr int COUNT = FINAL + 1;
-};
 
 struct BwdParams {
     MaskGeom g;
@@ -97,308 +54,23 @@ struct BwdParams {
     unsigned long long timeout_ns;
 };
 
-// Barrier over the 128 gradient threads that also ANDs a predicate across them,
-// so that all four warps take the same abort decision.
-__device__ __forceinline__ bool sync_and_128(bool pred)
+// Barrier over one gradient warpgroup (named barrier `id`, 128 threads).
+__device__ __forceinline__ void sync_wg(uint32_t id) { asm volatile("barrier.sync %0, 128;" ::"r"(id) : "memory"); }
+
+// The same barrier, also ANDing a predicate across the warpgroup, so that its
+// four warps take the same abort decision.
+__device__ __forceinline__ bool sync_and_wg(uint32_t id, bool pred)
 {
     uint32_t out;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 p, %1, 0;\n\t"
-        "barrier.red.and.pred q, 1, 128, p;\n\t"
+        "barrier.red.and.pred q, %2, 128, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(out)
-        : "r"(static_cast<uint32_t>(pred))
+        : "r"(static_cast<uint32_t>(pred)), "r"(id)
         : "memory");
     return out != 0;
-}
-
-template <int D, bool TRANS>
-__global__ void __launch_bounds__(BWD_THREADS, 1)
-    bwd_kernel(const __grid_constant__ CUtensorMap tmR0, const __grid_constant__ CUtensorMap tmR1,
-               const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY, const BwdParams p)
-{
-    using L = BLayout<D>;
-    using BB = BBars<L::XS, L::YS>;
-    static_assert(BB::COUNT * 8 + 8 <= 512, "barrier area");
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw_addr = smem_addr(smem_raw);
-    const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
-    uint8_t* smem = smem_raw + (sbase - raw_addr);
-    const uint32_t sR0 = sbase + L::R0_OFF, sR1 = sbase + L::R1_OFF, sX = sbase + L::X_OFF, sY = sbase + L::Y_OFF;
-    const uint32_t bars = sbase + L::BAR_OFF;
-    auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::BAR_OFF + 8 * BB::COUNT);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::BAR_OFF + 8 * BB::COUNT + 4);
-    float* stat = reinterpret_cast<float*>(smem + L::STAT_OFF);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;  // tb: query tile (dQ) or key tile (dK/dV)
-    const int bh = b * p.H + h;
-    const int n = p.g.n;
-    WaitCtl wc{abort_flag, p.err, p.timeout_ns};
-
-    if (threadIdx.x == 0) {
-        *abort_flag = *reinterpret_cast<volatile int*>(p.err) != 0 ? 1 : 0;
-        for (int i = 0; i < BB::COUNT; ++i)
-            mbar_init(bar(i), (i == BB::DS_FULL || i == BB::DS_FULL + 1) ? 128u : 1u);
-        fence_barrier_init();
-        fence_proxy_async_smem();
-    }
-    if (warp == 5) {
-        tmem_alloc(smem_addr(tmem_slot), BWD_TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const bool skip = *abort_flag != 0;
-    const int start = p.ptr[tb];
-    const int len = skip ? 0 : p.ptr[tb + 1] - start;
-    const int G = 2 * len;  // steps: two 64-row halves per walked tile
-
-    if (warp == 4) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0 && G > 0) {
-            mbar_arrive_expect_tx(bar(BB::RES_FULL), 2 * L::R_BYTES);
-            for (int c = 0; c < L::CHUNKS; ++c) {
-                tma_load_3d(sR0 + c * L::R_CHUNK_BYTES, &tmR0, bar(BB::RES_FULL), c * 64, tb * TILE, bh);
-                tma_load_3d(sR1 + c * L::R_CHUNK_BYTES, &tmR1, bar(BB::RES_FULL), c * 64, tb * TILE, bh);
-            }
-            int x_issued = 0, y_issued = 0;
-            for (int g = 0; g < G; ++g) {
-                const int row0 = p.idx[start + (g >> 1)] * TILE + (g & 1) * HALF;
-                const int xs = g % L::XS, ys = g % L::YS;
-                if (g >= L::XS && !mbar_wait(bar(BB::X_EMPTY + xs), ((g / L::XS) - 1) & 1, wc, BSITE_X_EMPTY))
-                    break;
-                mbar_arrive_expect_tx(bar(BB::X_FULL + xs), L::H_BYTES);
-                for (int c = 0; c < L::CHUNKS; ++c)
-                    tma_load_3d(sX + xs * L::H_BYTES + c * L::H_CHUNK_BYTES, &tmX, bar(BB::X_FULL + xs), c * 64,
-                                row0, bh);
-                x_issued = g + 1;
-                if (g >= L::YS && !mbar_wait(bar(BB::Y_EMPTY + ys), ((g / L::YS) - 1) & 1, wc, BSITE_Y_EMPTY))
-                    break;
-                mbar_arrive_expect_tx(bar(BB::Y_FULL + ys), L::H_BYTES);
-                for (int c = 0; c < L::CHUNKS; ++c)
-                    tma_load_3d(sY + ys * L::H_BYTES + c * L::H_CHUNK_BYTES, &tmY, bar(BB::Y_FULL + ys), c * 64,
-                                row0, bh);
-                y_issued = g + 1;
-            }
-            drain_wait(bar(BB::RES_FULL), 0, p.timeout_ns);
-            for (int g = max(0, x_issued - L::XS); g < x_issued; ++g)
-                drain_wait(bar(BB::X_FULL + g % L::XS), (g / L::XS) & 1, p.timeout_ns);
-            for (int g = max(0, y_issued - L::YS); g < y_issued; ++g)
-                drain_wait(bar(BB::Y_FULL + g % L::YS), (g / L::YS) & 1, p.timeout_ns);
-        }
-    } else if (warp == 5) {
-        // ----------------------------------------------------------------- MMA
-        if (lane == 0 && G > 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, HALF, 0, 0);  // A, B K-major, N = 64
-            constexpr uint32_t idesc_acc = idesc_bf16_f32(TILE, D, 0, 1);   // A from TMEM, B MN-major
-            // D[col] = A(resident 128 x d) * B(64-row half)^T over d.
-            auto mma_s = [&](uint32_t col, uint32_t a, uint32_t b2) {
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss(tmem + col,
-                           smem_desc_sw128(a + (kk >> 2) * L::R_CHUNK_BYTES + (kk & 3) * 32, 16, 1024),
-                           smem_desc_sw128(b2 + (kk >> 2) * L::H_CHUNK_BYTES + (kk & 3) * 32, 16, 1024), idesc_s,
-                           kk > 0 ? 1u : 0u);
-            };
-            // acc[col] += A(TMEM, 128 x 64 bf16 packed at acol) * B(64-row half, MN-major).
-            auto mma_acc = [&](uint32_t col, uint32_t acol, uint32_t b2, bool first) {
-#pragma unroll
-                for (int kk = 0; kk < HALF / 16; ++kk)
-                    mma_ts(tmem + col, tmem + acol + kk * 8, smem_desc_sw128(b2 + kk * 2048, L::H_CHUNK_BYTES, 1024),
-                           idesc_acc, (!first || kk > 0) ? 1u : 0u);
-            };
-            // gradient MMAs of step g (its dS / P in buffer g & 1), then release what it read
-            auto issue_acc = [&](int g) {
-                const int bf = g & 1, xs = g % L::XS, ys = g % L::YS;
-                const uint32_t x = sX + xs * L::H_BYTES, y = sY + ys * L::H_BYTES;
-                if (!TRANS) {
-                    mma_acc(COL_ACC0, s_col(bf), x, g == 0);   // dQ += dS K
-                } else {
-                    mma_acc(COL_ACC1, s_col(bf), y, g == 0);   // dV += P^T dO
-                    mma_acc(COL_ACC0, dp_col(bf), x, g == 0);  // dK += dS^T Q
-                }
-                mma_commit(bar(BB::ACC_DONE + bf));
-                mma_commit(bar(BB::X_EMPTY + xs));
-                if (TRANS)
-                    mma_commit(bar(BB::Y_EMPTY + ys));
-            };
-            bool ok = mbar_wait(bar(BB::RES_FULL), 0, wc, BSITE_RES);
-            tc_fence_after();
-            int acc_issued = 0;
-            for (int g = 0; ok && g < G; ++g) {
-                const int bf = g & 1, xs = g % L::XS, ys = g % L::YS;
-                if (!(ok = mbar_wait(bar(BB::X_FULL + xs), (g / L::XS) & 1, wc, BSITE_X_FULL)) ||
-                    !(ok = mbar_wait(bar(BB::Y_FULL + ys), (g / L::YS) & 1, wc, BSITE_Y_FULL)))
-                    break;
-                // S and dP of this step overwrite buffer bf, which the gradient
-                // MMAs of step g - 2 read; MMAs into different accumulators are
-                // not ordered, so wait for those first.
-                if (g >= 2 && !(ok = mbar_wait(bar(BB::ACC_DONE + bf), ((g - 2) >> 1) & 1, wc, BSITE_ACC)))
-                    break;
-                tc_fence_after();
-                mma_s(s_col(bf), sR0, sX + xs * L::H_BYTES);   // S = Q K^T, or S^T = K Q^T
-                mma_s(dp_col(bf), sR1, sY + ys * L::H_BYTES);  // dP = dO V^T, or dP^T = V dO^T
-                mma_commit(bar(BB::S_FULL + bf));
-                if (!TRANS)
-                    mma_commit(bar(BB::Y_EMPTY + ys));  // V half no longer needed
-                if (g >= 1) {
-                    if (!(ok = mbar_wait(bar(BB::DS_FULL + (bf ^ 1)), ((g - 1) >> 1) & 1, wc, BSITE_DS_FULL)))
-                        break;
-                    tc_fence_after();
-                    issue_acc(g - 1);
-                    acc_issued = g;
-                }
-            }
-            if (ok && acc_issued == G - 1) {
-                if (mbar_wait(bar(BB::DS_FULL + ((G - 1) & 1)), ((G - 1) >> 1) & 1, wc, BSITE_DS_FULL)) {
-                    tc_fence_after();
-                    issue_acc(G - 1);
-                }
-            }
-            mma_commit(bar(BB::FINAL));
-            drain_wait(bar(BB::FINAL), 0, p.timeout_ns);
-        }
-    } else {
-        // ------------------------------------------------------ gradient warps
-        const int t = threadIdx.x;  // == TMEM lane: query row (dQ) or key row (dK/dV) of the tile
-        const int row = tb * TILE + t;
-        const bool row_valid = row < n;
-        const int rf = row_valid ? row / p.g.s : 0, rp = row_valid ? row % p.g.s : 0;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        const bool tail = (n % TILE) != 0;
-        // per-row statistics of a query row (dQ pass)
-        const float row_l2 = (!TRANS && row_valid) ? p.lse[static_cast<size_t>(bh) * n + row] * LOG2E : 0.f;
-        const float row_d = (!TRANS && row_valid) ? p.Dv[static_cast<size_t>(bh) * n + row] : 0.f;
-        bool ok = true;
-        uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
-        bool masked = false;
-        for (int g = 0; g < G; ++g) {
-            const int j = g >> 1, half = g & 1, bf = g & 1;
-            const int other = p.idx[start + j];  // key tile (dQ) or query tile (dK/dV)
-            float* st_l2 = stat + bf * 2 * HALF;
-            float* st_d = st_l2 + HALF;
-            if (TRANS) {
-                // statistics of the step's 64 query columns; columns >= n get
-                // L = +inf so their P is exactly 0
-                const int q = other * TILE + half * HALF + (t & (HALF - 1));
-                if (t < HALF)
-                    st_l2[t] = q < n ? p.lse[static_cast<size_t>(bh) * n + q] * LOG2E : INFINITY;
-                else
-                    st_d[t - HALF] = q < n ? p.Dv[static_cast<size_t>(bh) * n + q] : 0.f;
-            }
-            if (half == 0) {
-                const bool partial = p.flag[start + j] != RA_TILE_FULL;
-                const bool use_family = p.mode == RA_MODE_TOKEN_EXACT && partial;
-                masked = use_family || (!TRANS && tail && other == p.nb - 1);
-                mk[0] = mk[1] = mk[2] = mk[3] = ~0u;
-                if (masked) {
-                    if (use_family && row_valid) {
-                        if (!TRANS)
-                            row_keep_mask(p.g, rf, rp, other * TILE, mk[0], mk[1], mk[2], mk[3]);
-                        else
-                            col_keep_mask(p.g, rf, rp, other * TILE, mk[0], mk[1], mk[2], mk[3]);
-                    } else if (!TRANS) {
-                        const int valid_cols = min(TILE, n - other * TILE);
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const int v = valid_cols - 32 * c;
-                            mk[c] = v >= 32 ? 0xFFFFFFFFu : (v <= 0 ? 0u : ((1u << v) - 1u));
-                        }
-                    }
-                }
-            }
-            ok = mbar_wait(bar(BB::S_FULL + bf), (g >> 1) & 1, wc, BSITE_S_FULL);
-            // one decision for all 128 threads; also publishes the staged statistics
-            ok = TRANS ? sync_and_128(ok) : __all_sync(0xFFFFFFFFu, ok);
-            if (!ok)
-                break;
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t sv[32], dv[32];
-                tmem_ld32(lane_base + s_col(bf) + c * 32, sv);
-                tmem_ld32(lane_base + dp_col(bf) + c * 32, dv);
-                tmem_wait_ld();
-                const uint32_t mword = half ? (c ? mk[3] : mk[2]) : (c ? mk[1] : mk[0]);
-                uint32_t pk[16], dk[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float pe[2], ds[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int col = c * 32 + e + u;
-                        const bool keep = !masked || ((mword >> (e + u)) & 1u);
-                        const float l2 = TRANS ? st_l2[col] : row_l2;
-                        const float dd = TRANS ? st_d[col] : row_d;
-                        const float x = fmaf(__uint_as_float(sv[e + u]), p.scale_log2, -l2);
-                        pe[u] = keep ? fast_exp2(x) : 0.f;
-                        ds[u] = pe[u] * (__uint_as_float(dv[e + u]) - dd);
-                    }
-                    pk[e >> 1] = pack_bf16(pe[0], pe[1]);
-                    dk[e >> 1] = pack_bf16(ds[0], ds[1]);
-                }
-                // Written over columns already read (chunk c goes to columns 16 c .. 16 c + 15).
-                if (!TRANS) {
-                    tmem_st16(lane_base + s_col(bf) + c * 16, dk);   // dS for dQ += dS K
-                } else {
-                    tmem_st16(lane_base + s_col(bf) + c * 16, pk);   // P^T for dV += P^T dO
-                    tmem_st16(lane_base + dp_col(bf) + c * 16, dk);  // dS^T for dK += dS^T Q
-                }
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(BB::DS_FULL + bf));
-        }
-        // ------------------------------------------------------------ epilogue
-        if (G > 0 && ok)
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(BB::FINAL), 0, wc, BSITE_FINAL));
-        tc_fence_after();
-        // tcgen05.ld is warp-collective: every lane loads, only rows < n store
-        if (__all_sync(0xFFFFFFFFu, ok && !*abort_flag)) {
-#pragma unroll 1
-            for (int which = 0; which < (TRANS ? 2 : 1); ++which) {
-                __nv_bfloat16* dst_row = (which == 0 ? p.out0 : p.out1) + (static_cast<size_t>(bh) * n + row) * D;
-                const float mul = which == 0 ? p.scale : 1.f;  // dQ, dK carry the softmax scale; dV does not
-                const uint32_t col0 = which == 0 ? COL_ACC0 : COL_ACC1;
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    if (G > 0) {
-                        tmem_ld32(lane_base + col0 + c * 32, o);
-                        tmem_wait_ld();
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            o[e] = 0u;
-                    }
-                    uint4 v[4];
-                    uint32_t* w = reinterpret_cast<uint32_t*>(v);
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2)
-                        w[e >> 1] = pack_bf16(__uint_as_float(o[e]) * mul, __uint_as_float(o[e + 1]) * mul);
-                    if (row_valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            dst[u] = v[u];
-                    }
-                }
-            }
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 5) {
-        __syncwarp();
-        tmem_dealloc(tmem, BWD_TMEM_COLS);
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -703,6 +375,338 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// dK / dV kernel with 128-query steps (N = 128 products).  One CTA per key
+// tile walks the transposed block-CSR.  TMEM (512 columns) holds S^T (0),
+// dP^T (128; dS^T is packed back over its first half), dK (256) and dV (384),
+// so P^T, the A operand of dV += P^T dO, goes to shared memory in the
+// 128-byte-swizzled K-major layout.  Per step j the MMA warp issues S^T_{j+1}
+// as soon as the gradient warps have loaded S^T_j and dP^T_j into registers,
+// then dK_j and dV_j, then dP^T_{j+1} once dK_j (which reads dS^T from the
+// dP^T columns) has completed; dV_j runs meanwhile.  320 threads: two
+// gradient warpgroups (query columns 64 wg .. 64 wg + 63 of each step), warp
+// 8 issues the TMA loads, warp 9 the MMAs.
+constexpr int KV_THREADS = 320, KV_GRAD_THREADS = 256, KV_PRODUCER_WARP = 8, KV_MMA_WARP = 9;
+constexpr uint32_t KV_COL_S = 0, KV_COL_DP = 128, KV_COL_DK = 256, KV_COL_DV = 384;
+
+template <int D>
+struct KvLayout {
+    static constexpr int CHUNKS = D / 64;
+    static constexpr int CHUNK_BYTES = TILE * 128;           // 128 rows x 128 bytes
+    static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;  // a 128 x d tile
+    static constexpr int PT_BYTES = 2 * CHUNK_BYTES;         // P^T: 128 keys x 128 queries bf16
+    static constexpr int QS = D == 64 ? 3 : 2;                // Q tile ring
+    static constexpr int OS = D == 64 ? 3 : 2;                // dO tile ring
+    static constexpr int K_OFF = 0, V_OFF = TILE_BYTES;
+    static constexpr int Q_OFF = 2 * TILE_BYTES;
+    static constexpr int DO_OFF = Q_OFF + QS * TILE_BYTES;
+    static constexpr int PT_OFF = DO_OFF + OS * TILE_BYTES;
+    static constexpr int STAT_OFF = PT_OFF + PT_BYTES;        // [L2, D][128] floats
+    static constexpr int BAR_OFF = STAT_OFF + 2 * TILE * 4;
+    static constexpr int SMEM_NEEDED = BAR_OFF + 256 + 1024;
+    static constexpr int SMEM_BYTES = SMEM_NEEDED > 120 * 1024 ? SMEM_NEEDED : 120 * 1024;
+    static_assert(SMEM_NEEDED <= 232448, "shared memory");
+};
+
+template <int QS, int OS>
+struct KvBars {
+    static constexpr int RES_FULL = 0;
+    static constexpr int Q_FULL = 1;
+    static constexpr int Q_EMPTY = Q_FULL + QS;
+    static constexpr int O_FULL = Q_EMPTY + QS;
+    static constexpr int O_EMPTY = O_FULL + OS;
+    static constexpr int S_FULL = O_EMPTY + OS;  // S^T_j and dP^T_j complete (and every earlier MMA)
+    static constexpr int S_FREE = S_FULL + 1;    // the gradient warps have loaded S^T_j and dP^T_j
+    static constexpr int DS_FULL = S_FREE + 1;   // P^T_j (shared memory) and dS^T_j (TMEM) written
+    static constexpr int DK_DONE = DS_FULL + 1;  // dK += dS^T_j Q_j complete
+    static constexpr int FINAL = DK_DONE + 1;
+    static constexpr int COUNT = FINAL + 1;
+};
+
+template <int D>
+__global__ void __launch_bounds__(KV_THREADS, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                    const BwdParams p)
+{
+    using L = KvLayout<D>;
+    using BB = KvBars<L::QS, L::OS>;
+    static_assert(BB::COUNT * 8 + 8 <= 256, "barrier area");
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_addr(smem_raw);
+    const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (sbase - raw_addr);
+    const uint32_t sK = sbase + L::K_OFF, sV = sbase + L::V_OFF, sQ = sbase + L::Q_OFF, sO = sbase + L::DO_OFF;
+    const uint32_t sPT = sbase + L::PT_OFF;
+    const uint32_t bars = sbase + L::BAR_OFF;
+    auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::BAR_OFF + 8 * BB::COUNT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::BAR_OFF + 8 * BB::COUNT + 4);
+    float* st_l2 = reinterpret_cast<float*>(smem + L::STAT_OFF);
+    float* st_d = st_l2 + TILE;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int bh = b * p.H + h;
+    const int n = p.g.n;
+    WaitCtl wc{abort_flag, p.err, p.timeout_ns};
+
+    if (threadIdx.x == 0) {
+        *abort_flag = *reinterpret_cast<volatile int*>(p.err) != 0 ? 1 : 0;
+        for (int i = 0; i < BB::COUNT; ++i) {
+            const bool grad = i == BB::S_FREE || i == BB::DS_FULL;
+            mbar_init(bar(i), grad ? static_cast<uint32_t>(KV_GRAD_THREADS) : 1u);
+        }
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == KV_MMA_WARP) {
+        tmem_alloc(smem_addr(tmem_slot), BWD_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const bool skip = *abort_flag != 0;
+    const int start = p.ptr[kb];
+    const int len = skip ? 0 : p.ptr[kb + 1] - start;
+
+    if (warp == KV_PRODUCER_WARP) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0 && len > 0) {
+            mbar_arrive_expect_tx(bar(BB::RES_FULL), 2 * L::TILE_BYTES);
+            for (int c = 0; c < L::CHUNKS; ++c) {
+                tma_load_3d(sK + c * L::CHUNK_BYTES, &tmK, bar(BB::RES_FULL), c * 64, kb * TILE, bh);
+                tma_load_3d(sV + c * L::CHUNK_BYTES, &tmV, bar(BB::RES_FULL), c * 64, kb * TILE, bh);
+            }
+            int q_issued = 0, o_issued = 0;
+            for (int j = 0; j < len; ++j) {
+                const int row0 = p.idx[start + j] * TILE;
+                const int qs = j % L::QS, os = j % L::OS;
+                if (j >= L::QS && !mbar_wait(bar(BB::Q_EMPTY + qs), ((j / L::QS) - 1) & 1, wc, BSITE_X_EMPTY))
+                    break;
+                mbar_arrive_expect_tx(bar(BB::Q_FULL + qs), L::TILE_BYTES);
+                for (int c = 0; c < L::CHUNKS; ++c)
+                    tma_load_3d(sQ + qs * L::TILE_BYTES + c * L::CHUNK_BYTES, &tmQ, bar(BB::Q_FULL + qs), c * 64, row0,
+                                bh);
+                q_issued = j + 1;
+                if (j >= L::OS && !mbar_wait(bar(BB::O_EMPTY + os), ((j / L::OS) - 1) & 1, wc, BSITE_Y_EMPTY))
+                    break;
+                mbar_arrive_expect_tx(bar(BB::O_FULL + os), L::TILE_BYTES);
+                for (int c = 0; c < L::CHUNKS; ++c)
+                    tma_load_3d(sO + os * L::TILE_BYTES + c * L::CHUNK_BYTES, &tmDO, bar(BB::O_FULL + os), c * 64,
+                                row0, bh);
+                o_issued = j + 1;
+            }
+            drain_wait(bar(BB::RES_FULL), 0, p.timeout_ns);
+            for (int j = max(0, q_issued - L::QS); j < q_issued; ++j)
+                drain_wait(bar(BB::Q_FULL + j % L::QS), (j / L::QS) & 1, p.timeout_ns);
+            for (int j = max(0, o_issued - L::OS); j < o_issued; ++j)
+                drain_wait(bar(BB::O_FULL + j % L::OS), (j / L::OS) & 1, p.timeout_ns);
+        }
+    } else if (warp == KV_MMA_WARP) {
+        // ----------------------------------------------------------------- MMA
+        if (lane == 0 && len > 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, TILE, 0, 0);  // A, B K-major, N = 128
+            constexpr uint32_t idesc_acc = idesc_bf16_f32(TILE, D, 0, 1);   // A K-major, B MN-major
+            // D[col] = A(resident 128 x d) * B(128-row tile)^T over d.
+            auto mma_s = [&](uint32_t col, uint32_t a, uint32_t b2) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
+                    mma_ss(tmem + col, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b2 + off, 16, 1024),
+                           idesc_s, kk > 0 ? 1u : 0u);
+                }
+            };
+            // dK += dS^T_j Q_j: dS^T packed by the warpgroups, queries 16 kk .. 16 kk + 15
+            // at columns 64 (kk / 4) + 8 (kk % 4) of the dP^T buffer.
+            auto issue_dk = [&](int j) {
+                const int qs = j % L::QS;
+                const uint32_t qbase = sQ + qs * L::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < TILE / 16; ++kk)
+                    mma_ts(tmem + KV_COL_DK, tmem + KV_COL_DP + (kk >> 2) * 64 + (kk & 3) * 8,
+                           smem_desc_sw128(qbase + kk * 2048, L::CHUNK_BYTES, 1024), idesc_acc,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar(BB::DK_DONE));
+                mma_commit(bar(BB::Q_EMPTY + qs));
+            };
+            // dV += P^T_j dO_j: P^T from shared memory (K-major over the queries).
+            auto issue_dv = [&](int j) {
+                const int os = j % L::OS;
+                const uint32_t obase = sO + os * L::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < TILE / 16; ++kk)
+                    mma_ss(tmem + KV_COL_DV, smem_desc_sw128(sPT + (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32, 16, 1024),
+                           smem_desc_sw128(obase + kk * 2048, L::CHUNK_BYTES, 1024), idesc_acc,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar(BB::O_EMPTY + os));
+            };
+            bool ok = mbar_wait(bar(BB::RES_FULL), 0, wc, BSITE_RES) &&
+                      mbar_wait(bar(BB::Q_FULL), 0, wc, BSITE_X_FULL);
+            if (ok) {
+                tc_fence_after();
+                mma_s(KV_COL_S, sK, sQ);
+                ok = mbar_wait(bar(BB::O_FULL), 0, wc, BSITE_Y_FULL);
+            }
+            if (ok) {
+                tc_fence_after();
+                mma_s(KV_COL_DP, sV, sO);
+                mma_commit(bar(BB::S_FULL));
+            }
+            for (int j = 0; ok && j < len; ++j) {
+                const int jn = j + 1;
+                if (jn < len) {
+                    // S^T_{j+1} over S^T_j, which the gradient warps have loaded
+                    if (!(ok = mbar_wait(bar(BB::Q_FULL + jn % L::QS), (jn / L::QS) & 1, wc, BSITE_X_FULL)) ||
+                        !(ok = mbar_wait(bar(BB::S_FREE), j & 1, wc, BSITE_S_FULL)))
+                        break;
+                    tc_fence_after();
+                    mma_s(KV_COL_S, sK, sQ + (jn % L::QS) * L::TILE_BYTES);
+                }
+                if (!(ok = mbar_wait(bar(BB::DS_FULL), j & 1, wc, BSITE_DS_FULL)))
+                    break;
+                tc_fence_after();
+                issue_dk(j);
+                issue_dv(j);
+                if (jn < len) {
+                    // dP^T_{j+1} over the dS^T_j that dK_j read: wait for dK_j only
+                    // (MMAs into different accumulators are not ordered); dV_j runs on
+                    if (!(ok = mbar_wait(bar(BB::O_FULL + jn % L::OS), (jn / L::OS) & 1, wc, BSITE_Y_FULL)) ||
+                        !(ok = mbar_wait(bar(BB::DK_DONE), j & 1, wc, BSITE_ACC)))
+                        break;
+                    tc_fence_after();
+                    mma_s(KV_COL_DP, sV, sO + (jn % L::OS) * L::TILE_BYTES);
+                    mma_commit(bar(BB::S_FULL));
+                }
+            }
+            mma_commit(bar(BB::FINAL));
+            drain_wait(bar(BB::FINAL), 0, p.timeout_ns);
+        }
+    } else {
+        // ------------------------------------------------------ gradient warps
+        const int wg = warp >> 2;            // warpgroup: query columns 64 wg .. 64 wg + 63 of each step
+        const int t = threadIdx.x & 127;     // == TMEM lane: key row of the tile
+        const int row = kb * TILE + t;
+        const bool row_valid = row < n;
+        const int rf = row_valid ? row / p.g.s : 0, rp = row_valid ? row % p.g.s : 0;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const uint32_t my_col = 64u * static_cast<uint32_t>(wg);
+        const uint32_t wg_bar = 1u + static_cast<uint32_t>(wg);
+        // this thread's row of P^T (K-major, 128-byte swizzle): chunk wg holds its 64 queries
+        uint8_t* pt_row = smem + L::PT_OFF + wg * L::CHUNK_BYTES + t * 128;
+        bool ok = true;
+        for (int j = 0; j < len; ++j) {
+            const int qb = p.idx[start + j];
+            const bool masked = p.mode == RA_MODE_TOKEN_EXACT && p.flag[start + j] != RA_TILE_FULL;
+            uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
+            if (masked && row_valid)
+                col_keep_mask(p.g, rf, rp, qb * TILE, mk[0], mk[1], mk[2], mk[3]);
+            // statistics of the step's query columns (this warpgroup's 64): lse
+            // (log2 units; +inf beyond n, so P is exactly 0 there) and D
+            sync_wg(wg_bar);  // the previous step's readers are done
+            if (t < 64) {
+                const int q = qb * TILE + static_cast<int>(my_col) + t;
+                st_l2[my_col + t] = q < n ? p.lse[static_cast<size_t>(bh) * n + q] * LOG2E : INFINITY;
+            } else {
+                const int q = qb * TILE + static_cast<int>(my_col) + t - 64;
+                st_d[my_col + t - 64] = q < n ? p.Dv[static_cast<size_t>(bh) * n + q] : 0.f;
+            }
+            ok = mbar_wait(bar(BB::S_FULL), j & 1, wc, BSITE_S_FULL);
+            // one decision per warpgroup; also publishes its staged statistics
+            ok = sync_and_wg(wg_bar, ok);
+            if (!ok)
+                break;
+            tc_fence_after();
+            // S^T first, then release it for S^T_{j+1}; dP^T stays until dK_j has
+            // read the dS^T packed over it
+            uint32_t sv[2][32];
+            tmem_ld32(lane_base + KV_COL_S + my_col, sv[0]);
+            tmem_ld32(lane_base + KV_COL_S + my_col + 32, sv[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar(BB::S_FREE));
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t dvc[32];
+                tmem_ld32(lane_base + KV_COL_DP + my_col + c * 32, dvc);
+                tmem_wait_ld();
+                const uint32_t mword = wg ? (c ? mk[3] : mk[2]) : (c ? mk[1] : mk[0]);
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float pe[2], ds[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int col = static_cast<int>(my_col) + c * 32 + e + u;
+                        const bool keep = !masked || ((mword >> (e + u)) & 1u);
+                        const float x = fmaf(__uint_as_float(sv[c][e + u]), p.scale_log2, -st_l2[col]);
+                        pe[u] = keep ? fast_exp2(x) : 0.f;
+                        ds[u] = pe[u] * (__uint_as_float(dvc[e + u]) - st_d[col]);
+                    }
+                    pk[e >> 1] = pack_bf16(pe[0], pe[1]);
+                    dk[e >> 1] = pack_bf16(ds[0], ds[1]);
+                }
+                // P^T: 16-byte units 4 c .. 4 c + 3 of the row, at unit ^ (row % 8)
+#pragma unroll
+                for (int uu = 0; uu < 4; ++uu) {
+                    const int unit = 4 * c + uu;
+                    *reinterpret_cast<uint4*>(pt_row + ((unit ^ (t & 7)) * 16)) =
+                        make_uint4(pk[4 * uu], pk[4 * uu + 1], pk[4 * uu + 2], pk[4 * uu + 3]);
+                }
+                // dS^T packed over dP^T columns this warpgroup has already loaded
+                tmem_st16(lane_base + KV_COL_DP + my_col + c * 16, dk);
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();  // P^T is read by the tensor cores
+            tc_fence_before();
+            mbar_arrive(bar(BB::DS_FULL));
+        }
+        // ------------------------------------------------------------ epilogue
+        // warpgroup 0 stores dK (times the softmax scale), warpgroup 1 dV
+        if (len > 0 && ok)
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(BB::FINAL), 0, wc, BSITE_FINAL));
+        tc_fence_after();
+        if (__all_sync(0xFFFFFFFFu, ok && !*abort_flag)) {
+            __nv_bfloat16* dst_row = (wg ? p.out1 : p.out0) + (static_cast<size_t>(bh) * n + row) * D;
+            const float mul = wg ? 1.f : p.scale;
+            const uint32_t col0 = wg ? KV_COL_DV : KV_COL_DK;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                if (len > 0) {
+                    tmem_ld32(lane_base + col0 + c * 32, o);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        o[e] = 0u;
+                }
+                uint4 v[4];
+                uint32_t* w = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+                for (int e = 0; e < 32; e += 2)
+                    w[e >> 1] = pack_bf16(__uint_as_float(o[e]) * mul, __uint_as_float(o[e + 1]) * mul);
+                if (row_valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        dst[u] = v[u];
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == KV_MMA_WARP) {
+        __syncwarp();
+        tmem_dealloc(tmem, BWD_TMEM_COLS);
+    }
+}
+
 // D[r] = <dO[r], O[r]> over d, one warp per row.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_dot_kernel(const __nv_bfloat16* __restrict__ O,
@@ -728,21 +732,21 @@ __global__ void __launch_bounds__(256) bwd_dot_kernel(const __nv_bfloat16* __res
     }
 }
 
-template <int D, bool TRANS>
-ra_status launch_bwd(const CUtensorMap& r0, const CUtensorMap& r1, const CUtensorMap& x, const CUtensorMap& y,
-                     const BwdParams& p, int B, cudaStream_t cs)
+template <int D>
+ra_status launch_dkdv(const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& q, const CUtensorMap& dO,
+                      const BwdParams& p, int B, cudaStream_t cs)
 {
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(bwd_kernel<D, TRANS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        BLayout<D>::SMEM_BYTES);
+        attr_err = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        KvLayout<D>::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess)
-        return cuda_fail(attr_err, "cudaFuncSetAttribute(bwd_kernel)");
+        return cuda_fail(attr_err, "cudaFuncSetAttribute(bwd_dkdv_kernel)");
     dim3 grid(p.nb, p.H, B);
-    bwd_kernel<D, TRANS><<<grid, BWD_THREADS, BLayout<D>::SMEM_BYTES, cs>>>(r0, r1, x, y, p);
-    return cuda_fail(cudaGetLastError(), "bwd_kernel launch");
+    bwd_dkdv_kernel<D><<<grid, KV_THREADS, KvLayout<D>::SMEM_BYTES, cs>>>(k, v, q, dO, p);
+    return cuda_fail(cudaGetLastError(), "bwd_dkdv_kernel launch");
 }
 
 template <int D>
@@ -775,11 +779,9 @@ ra_status run_bwd(const void* Q, const void* K, const void* V, const void* O, co
     ra_status st = cuda_fail(cudaGetLastError(), "bwd_dot_kernel launch");
     if (st != RA_OK)
         return st;
-    // resident tiles: 128-row boxes; walked tiles: 64-row halves
-    CUtensorMap rq, rk, rv, rdo, hq, hdo;
+    CUtensorMap rq, rk, rv, rdo;  // 128-row boxes
     if ((st = make_map(&rq, Q, BH, n, D, TILE)) != RA_OK || (st = make_map(&rdo, dO, BH, n, D, TILE)) != RA_OK ||
-        (st = make_map(&rk, K, BH, n, D, TILE)) != RA_OK || (st = make_map(&rv, V, BH, n, D, TILE)) != RA_OK ||
-        (st = make_map(&hq, Q, BH, n, D, HALF)) != RA_OK || (st = make_map(&hdo, dO, BH, n, D, HALF)) != RA_OK)
+        (st = make_map(&rk, K, BH, n, D, TILE)) != RA_OK || (st = make_map(&rv, V, BH, n, D, TILE)) != RA_OK)
         return st;
     BwdParams p;
     std::memset(&p, 0, sizeof p);
@@ -802,13 +804,13 @@ ra_status run_bwd(const void* Q, const void* K, const void* V, const void* O, co
     p.out1 = nullptr;
     if ((st = launch_dq<D>(rq, rdo, rk, rv, p, B, cs)) != RA_OK)
         return st;
-    // dK, dV: key tiles over the transposed block-CSR; resident K, V; rings of Q, dO halves
+    // dK, dV: key tiles over the transposed block-CSR; resident K, V; rings of whole Q, dO tiles
     p.ptr = m->col_ptr;
     p.idx = m->row_idx;
     p.flag = m->tflag;
     p.out0 = static_cast<__nv_bfloat16*>(dK);
     p.out1 = static_cast<__nv_bfloat16*>(dV);
-    return launch_bwd<D, true>(rk, rv, hq, hdo, p, B, cs);
+    return launch_dkdv<D>(rk, rv, rq, rdo, p, B, cs);
 }
 
 }  // namespace
