@@ -275,10 +275,17 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
         const float row_l2 = row_valid ? p.lse[static_cast<size_t>(bh) * n + row] * LOG2E : 0.f;
         const float row_d = row_valid ? p.Dv[static_cast<size_t>(bh) * n + row] : 0.f;
         bool ok = true;
+        // CSR entry of the next step, loaded one step ahead of its use
+        int next_kb = len > 0 ? p.idx[start] : 0;
+        int next_flag = len > 0 ? p.flag[start] : 0;
         for (int j = 0; j < len; ++j) {
             const int bf = j & 1;
-            const int kb = p.idx[start + j];
-            const bool use_family = p.mode == RA_MODE_TOKEN_EXACT && p.flag[start + j] != RA_TILE_FULL;
+            const int kb = next_kb;
+            const bool use_family = p.mode == RA_MODE_TOKEN_EXACT && next_flag != RA_TILE_FULL;
+            if (j + 1 < len) {
+                next_kb = p.idx[start + j + 1];
+                next_flag = p.flag[start + j + 1];
+            }
             const bool masked = use_family || (tail && kb == p.nb - 1);
             uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
             if (masked) {
@@ -297,18 +304,20 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
             if (!ok)
                 break;
             tc_fence_after();
-            // dP first, then release the dP buffer for the next step's MMA
-            uint32_t dv[2][32];
+            // dP (and the first S chunk) first, then release the dP buffer for the
+            // next step's MMA; the second S chunk loads while the first is processed
+            uint32_t dv[2][32], sv[2][32];
             tmem_ld32(lane_base + DQ_COL_DP + my_col, dv[0]);
             tmem_ld32(lane_base + DQ_COL_DP + my_col + 32, dv[1]);
+            tmem_ld32(lane_base + dq_s_col(bf) + my_col, sv[0]);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar(BB::DP_FREE));
+            tmem_ld32(lane_base + dq_s_col(bf) + my_col + 32, sv[1]);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                uint32_t sv[32];
-                tmem_ld32(lane_base + dq_s_col(bf) + my_col + c * 32, sv);
-                tmem_wait_ld();
+                if (c == 1)
+                    tmem_wait_ld();
                 const uint32_t mword = wg ? (c ? mk[3] : mk[2]) : (c ? mk[1] : mk[0]);
                 uint32_t dk[16];
 #pragma unroll
@@ -317,7 +326,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const bool keep = !masked || ((mword >> (e + u)) & 1u);
-                        const float x = fmaf(__uint_as_float(sv[e + u]), p.scale_log2, -row_l2);
+                        const float x = fmaf(__uint_as_float(sv[c][e + u]), p.scale_log2, -row_l2);
                         const float pe = keep ? fast_exp2(x) : 0.f;
                         ds[u] = pe * (__uint_as_float(dv[c][e + u]) - row_d);
                     }
@@ -419,7 +428,8 @@ struct KvBars {
     static constexpr int S_FREE = S_FULL + 1;    // the gradient warps have loaded S^T_j and dP^T_j
     static constexpr int DS_FULL = S_FREE + 1;   // P^T_j (shared memory) and dS^T_j (TMEM) written
     static constexpr int DK_DONE = DS_FULL + 1;  // dK += dS^T_j Q_j complete
-    static constexpr int FINAL = DK_DONE + 1;
+    static constexpr int DV_DONE = DK_DONE + 1;  // dV += P^T_j dO_j complete (P^T may be overwritten)
+    static constexpr int FINAL = DV_DONE + 1;
     static constexpr int COUNT = FINAL + 1;
 };
 
@@ -541,6 +551,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                     mma_ss(tmem + KV_COL_DV, smem_desc_sw128(sPT + (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32, 16, 1024),
                            smem_desc_sw128(obase + kk * 2048, L::CHUNK_BYTES, 1024), idesc_acc,
                            (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar(BB::DV_DONE));
                 mma_commit(bar(BB::O_EMPTY + os));
             };
             bool ok = mbar_wait(bar(BB::RES_FULL), 0, wc, BSITE_RES) &&
@@ -569,10 +580,11 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                     break;
                 tc_fence_after();
                 issue_dk(j);
-                issue_dv(j);
                 if (jn < len) {
-                    // dP^T_{j+1} over the dS^T_j that dK_j read: wait for dK_j only
-                    // (MMAs into different accumulators are not ordered); dV_j runs on
+                    // dP^T_{j+1} over the dS^T_j that dK_j read: once dK_j has
+                    // completed (MMAs into different accumulators are not
+                    // ordered), and ahead of dV_j, so that the next step's
+                    // gradient warps start sooner
                     if (!(ok = mbar_wait(bar(BB::O_FULL + jn % L::OS), (jn / L::OS) & 1, wc, BSITE_Y_FULL)) ||
                         !(ok = mbar_wait(bar(BB::DK_DONE), j & 1, wc, BSITE_ACC)))
                         break;
@@ -580,6 +592,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                     mma_s(KV_COL_DP, sV, sO + (jn % L::OS) * L::TILE_BYTES);
                     mma_commit(bar(BB::S_FULL));
                 }
+                issue_dv(j);
             }
             mma_commit(bar(BB::FINAL));
             drain_wait(bar(BB::FINAL), 0, p.timeout_ns);
@@ -597,23 +610,34 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
         // this thread's row of P^T (K-major, 128-byte swizzle): chunk wg holds its 64 queries
         uint8_t* pt_row = smem + L::PT_OFF + wg * L::CHUNK_BYTES + t * 128;
         bool ok = true;
+        // Statistic of one query column of the step's (this warpgroup's 64):
+        // threads 0-63 the lse in log2 units (+inf beyond n, so P is exactly 0
+        // there), threads 64-127 D.  Loaded one step ahead of its use, with the
+        // CSR entry.
+        auto column_stat = [&](int qblock) -> float {
+            const int q = qblock * TILE + static_cast<int>(my_col) + (t & 63);
+            if (q >= n)
+                return t < 64 ? INFINITY : 0.f;
+            return t < 64 ? p.lse[static_cast<size_t>(bh) * n + q] * LOG2E : p.Dv[static_cast<size_t>(bh) * n + q];
+        };
+        int next_qb = len > 0 ? p.idx[start] : 0;
+        int next_flag = len > 0 ? p.flag[start] : 0;
+        float next_stat = len > 0 ? column_stat(next_qb) : 0.f;
         for (int j = 0; j < len; ++j) {
-            const int qb = p.idx[start + j];
-            const bool masked = p.mode == RA_MODE_TOKEN_EXACT && p.flag[start + j] != RA_TILE_FULL;
+            const int qb = next_qb;
+            const bool masked = p.mode == RA_MODE_TOKEN_EXACT && next_flag != RA_TILE_FULL;
+            const float stat = next_stat;
+            if (j + 1 < len) {
+                next_qb = p.idx[start + j + 1];
+                next_flag = p.flag[start + j + 1];
+                next_stat = column_stat(next_qb);
+            }
             uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
             if (masked && row_valid)
                 col_keep_mask(p.g, rf, rp, qb * TILE, mk[0], mk[1], mk[2], mk[3]);
-            // statistics of the step's query columns (this warpgroup's 64): lse
-            // (log2 units; +inf beyond n, so P is exactly 0 there) and D
-            sync_wg(wg_bar);  // the previous step's readers are done
-            if (t < 64) {
-                const int q = qb * TILE + static_cast<int>(my_col) + t;
-                st_l2[my_col + t] = q < n ? p.lse[static_cast<size_t>(bh) * n + q] * LOG2E : INFINITY;
-            } else {
-                const int q = qb * TILE + static_cast<int>(my_col) + t - 64;
-                st_d[my_col + t - 64] = q < n ? p.Dv[static_cast<size_t>(bh) * n + q] : 0.f;
-            }
-            ok = mbar_wait(bar(BB::S_FULL), j & 1, wc, BSITE_S_FULL);
+            sync_wg(wg_bar);  // the previous step's readers of the statistics are done
+            (t < 64 ? st_l2 : st_d)[my_col + (t & 63)] = stat;
+            ok = ok && mbar_wait(bar(BB::S_FULL), j & 1, wc, BSITE_S_FULL);
             // one decision per warpgroup; also publishes its staged statistics
             ok = sync_and_wg(wg_bar, ok);
             if (!ok)
@@ -621,33 +645,46 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
             tc_fence_after();
             // S^T first, then release it for S^T_{j+1}; dP^T stays until dK_j has
             // read the dS^T packed over it
-            uint32_t sv[2][32];
+            uint32_t sv[2][32], dv[2][32];
             tmem_ld32(lane_base + KV_COL_S + my_col, sv[0]);
             tmem_ld32(lane_base + KV_COL_S + my_col + 32, sv[1]);
+            tmem_ld32(lane_base + KV_COL_DP + my_col, dv[0]);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar(BB::S_FREE));
+            tmem_ld32(lane_base + KV_COL_DP + my_col + 32, dv[1]);  // lands while chunk 0 is processed
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                uint32_t dvc[32];
-                tmem_ld32(lane_base + KV_COL_DP + my_col + c * 32, dvc);
-                tmem_wait_ld();
+                if (c == 1)
+                    tmem_wait_ld();
+                const uint32_t (&dvc)[32] = dv[c];
                 const uint32_t mword = wg ? (c ? mk[3] : mk[2]) : (c ? mk[1] : mk[0]);
+                const float4* l2v = reinterpret_cast<const float4*>(st_l2 + my_col + c * 32);
+                const float4* dsv = reinterpret_cast<const float4*>(st_d + my_col + c * 32);
                 uint32_t pk[16], dk[16];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float pe[2], ds[2];
+                for (int e4 = 0; e4 < 32; e4 += 4) {
+                    const float4 l4 = l2v[e4 >> 2], d4 = dsv[e4 >> 2];  // same address in every lane
+                    const float lq[4] = {l4.x, l4.y, l4.z, l4.w}, dq[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float pe[4], ds[4];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int col = static_cast<int>(my_col) + c * 32 + e + u;
-                        const bool keep = !masked || ((mword >> (e + u)) & 1u);
-                        const float x = fmaf(__uint_as_float(sv[c][e + u]), p.scale_log2, -st_l2[col]);
+                    for (int u = 0; u < 4; ++u) {
+                        const int e = e4 + u;
+                        const bool keep = !masked || ((mword >> e) & 1u);
+                        const float x = fmaf(__uint_as_float(sv[c][e]), p.scale_log2, -lq[u]);
                         pe[u] = keep ? fast_exp2(x) : 0.f;
-                        ds[u] = pe[u] * (__uint_as_float(dvc[e + u]) - st_d[col]);
+                        ds[u] = pe[u] * (__uint_as_float(dvc[e]) - dq[u]);
                     }
-                    pk[e >> 1] = pack_bf16(pe[0], pe[1]);
-                    dk[e >> 1] = pack_bf16(ds[0], ds[1]);
+                    pk[e4 >> 1] = pack_bf16(pe[0], pe[1]);
+                    pk[(e4 >> 1) + 1] = pack_bf16(pe[2], pe[3]);
+                    dk[e4 >> 1] = pack_bf16(ds[0], ds[1]);
+                    dk[(e4 >> 1) + 1] = pack_bf16(ds[2], ds[3]);
                 }
+                // dV_{j-1} reads P^T_{j-1}: wait for it before the first overwrite.
+                // A failed wait is acted on at the next step's warpgroup barrier,
+                // so that the four warps leave the loop together.
+                if (c == 0 && j > 0)
+                    ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(BB::DV_DONE), (j - 1) & 1, wc, BSITE_ACC)) && ok;
                 // P^T: 16-byte units 4 c .. 4 c + 3 of the row, at unit ^ (row % 8)
 #pragma unroll
                 for (int uu = 0; uu < 4; ++uu) {
