@@ -204,7 +204,7 @@ def flops_per_call(info, c, mode, kind="fwd"):
     return (4.0 if kind == "fwd" else 10.0) * c["d"] * pairs * c["B"] * c["H"]
 
 
-def cpu_oracle_sample(name, mask, mode, c, target_s=15.0, seed_rank=0, kind="fwd"):
+def cpu_oracle_sample(name, mask, mode, c, target_s=15.0, seed_rank=0, kind="fwd", threads=None):
     """Time the oracle (as it stands) on a bounded sample of the workload: query
     rows of head 0 until about target_s seconds of CPU work.  Forward: the
     attention of each row (4 d FLOP per computed pair).  Backward: the dQ of each
@@ -212,6 +212,9 @@ def cpu_oracle_sample(name, mask, mode, c, target_s=15.0, seed_rank=0, kind="fwd
     Returns (TFLOP/s, threads, sample description)."""
     import oracle
     orc = oracle.default()
+    all_threads = orc.threads()
+    if threads:
+        orc.set_threads(threads)
     spec = oracle.spec_from(mask, c["f"], c["s"], c["grid"])
     n, d = c["f"] * c["s"], c["d"]
     shape = (1, 1, n, d)
@@ -237,12 +240,33 @@ def cpu_oracle_sample(name, mask, mode, c, target_s=15.0, seed_rank=0, kind="fwd
         flop += per_pair * float(nk.sum())
         done_rows += len(rows)
         nrows = min(nrows * 2, 1024)
+    used = orc.threads()
+    if threads:
+        orc.set_threads(all_threads)
     what = "attention" if kind == "fwd" else "dQ (with the S, O, dP it needs)"
     desc = (f"{what} of {done_rows} query rows of head 0 "
             f"({'kept tiles in full' if mode == 'block' else 'token-exact keys'}), "
             f"{int(flop / per_pair)} computed pairs, {elapsed:.1f} s, including the oracle's brute-force tile "
             f"flags of the rows' query tiles")
-    return flop / elapsed / 1e12, orc.threads(), desc
+    return flop / elapsed / 1e12, used, desc
+
+
+def cpu_oracle_extras(name, mask, mode, c, kind="fwd"):
+    """The oracle on one core (a short sample of the same rows) and its mask build
+    (brute-force tile counts of 8 query tiles, extrapolated to every tile)."""
+    import oracle
+    orc = oracle.default()
+    v1, _, desc1 = cpu_oracle_sample(name, mask, mode, c, target_s=4.0, kind=kind, threads=1)
+    spec = oracle.spec_from(mask, c["f"], c["s"], c["grid"])
+    nb = spec.nb
+    qbs = np.unique(np.linspace(0, nb - 1, num=min(8, nb)).astype(np.int32))
+    t0 = time.perf_counter()
+    orc.tile_counts(spec, qbs)
+    dt = time.perf_counter() - t0
+    return {"value_1core": v1, "sample_1core": desc1,
+            "mask_build_s_extrapolated": dt * nb / len(qbs),
+            "mask_build_sample": f"brute-force tile counts of {len(qbs)} of {nb} query tiles in {dt:.2f} s "
+                                 f"on {orc.threads()} threads, scaled to all {nb}"}
 
 
 def run_reference(args, c, mask):
@@ -583,6 +607,10 @@ def main():
     o = torch.empty_like(q)
     m = ra.build_mask(mask, c["f"], c["s"], c["grid"])
     info = m.info
+    # the mask is static: built once per shape, outside the timed region; timed here on its own
+    t_mb = time.perf_counter()
+    ra.build_mask(mask, c["f"], c["s"], c["grid"]).free()  # synchronises
+    mask_build_ms = (time.perf_counter() - t_mb) * 1e3
     bwd = args.pass_ == "bwd"
     flop = flops_per_call(info, c, args.mode, args.pass_)
     scale = 1.0 / math.sqrt(d)
@@ -654,6 +682,7 @@ def main():
                 "kernel": ("attn_fwd_kernel<%d>" % d) if not bwd else
                 ("ra_attention_bwd call: bwd_dot_kernel<%d> + bwd_kernel<%d, dQ> + bwd_kernel<%d, dK dV>" % (d, d, d)),
                 "flop_per_launch": flop,
+                "flop_executed_per_launch": flops_per_call(info, c, "block", args.pass_),
                 "algorithmic_bytes_per_launch": bytes_qkvo}
 
     # ---- end to end: host buffers through the C ABI (H2D + kernel + D2H per step)
@@ -743,6 +772,7 @@ def main():
     if world == 1 and not args.no_cpu_baseline:
         val, threads, desc = cpu_oracle_sample(args.workload, mask, args.mode, c, kind=args.pass_)
         cpu = {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+        cpu.update(cpu_oracle_extras(args.workload, mask, args.mode, c, kind=args.pass_))
 
     tile_total = info["nb"] ** 2
     line = {
@@ -760,8 +790,13 @@ def main():
             "kept_tiles": info["nnz"], "tile_sparsity": 1.0 - info["nnz"] / tile_total,
             "token_sparsity": 1.0 - info["kept_pairs"] / float(n) ** 2,
             "flop_definition": ("4*d" if not bwd else "10*d (S, dP, dQ, dK, dV)") +
-                               " per computed pair per head; block mode computes every valid pair of kept tiles",
+                               " per pair per head; block mode counts (and computes) every valid pair of the kept "
+                               "tiles; token-exact mode counts the kept pairs, and roofline.flop_executed_per_launch "
+                               "the pairs of the kept tiles the kernel executes",
         },
+        "launch_ms": {"median": float(np.median(launch_ms)), "min": float(np.min(launch_ms)),
+                      "p90": float(np.percentile(launch_ms, 90)), "launches": len(launch_ms)},
+        "mask_build_ms": mask_build_ms,
         "pct_of_peak": 100.0 * roofline["frac"],
         "roofline": roofline,
         "clocks": clk.summary(),

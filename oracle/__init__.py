@@ -112,6 +112,8 @@ def load_library(path: str):
     lib.oracle_attention_bwd.argtypes = [vp, vp, vp, vp, c_int, i64, c_int, P, c_int, ctypes.c_double, vp, vp, vp,
                                          vp]
     lib.oracle_attention_bwd.restype = None
+    lib.oracle_set_threads.argtypes = [c_int]
+    lib.oracle_set_threads.restype = None
     lib.oracle_attention_bwd_query_rows.argtypes = [vp, vp, vp, vp, c_int, i64, c_int, P, c_int, ctypes.c_double,
                                                     i64, vp, vp, vp, vp, vp, vp]
     lib.oracle_attention_bwd_query_rows.restype = None
@@ -139,6 +141,10 @@ class Oracle:
 
     def threads(self) -> int:
         return self.lib.oracle_threads()
+
+    def set_threads(self, n: int) -> None:
+        """Threads of the oracle's parallel loops from now on (timing only; results do not change)."""
+        self.lib.oracle_set_threads(int(n))
 
     def kept(self, spec: MaskSpec, q: int, key: int) -> int:
         sp = spec.c()

@@ -86,6 +86,17 @@ int oracle_threads(void)
 #endif
 }
 
+/* Threads the oracle's OpenMP loops use from now on (n >= 1). */
+void oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n >= 1)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 static long long or_abs(long long x) { return x < 0 ? -x : x; }
 
 /* floor(log2(x)) for x >= 1: position of the highest set bit. */
