@@ -1,0 +1,71 @@
+"""Host-side pieces of bench.py (CPU): FLOP definitions, the DRAM-traffic records
+and their source hashes, and the argument surface of the timed passes."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import bench as b
+    return b
+
+
+def test_flop_definitions(bench):
+    import synth
+    c = synth.CONFIGS["hunyuan108k"]
+    info = {"block_pairs": 1000, "kept_pairs": 600}
+    d, BH = c["d"], c["B"] * c["H"]
+    assert bench.flops_per_call(info, c, "block") == 4 * d * 1000 * BH
+    assert bench.flops_per_call(info, c, "token_exact") == 4 * d * 600 * BH
+    # the backward counts the five products S, dP, dQ, dK, dV: 2.5 times the forward
+    assert bench.flops_per_call(info, c, "block", "bwd") == 2.5 * bench.flops_per_call(info, c, "block")
+
+
+def test_traffic_records_follow_the_kernel_sources(bench, tmp_path, monkeypatch):
+    # the committed records parse, and each names the hash of its own kernel's sources
+    for kind in ("fwd", "bwd"):
+        path = os.path.join(ROOT, "profiles", f"attn_{kind}_traffic.txt")
+        assert os.path.exists(path), path
+        for rel in bench.ATTN_SOURCES[kind]:
+            assert os.path.exists(os.path.join(ROOT, rel)), rel
+    assert bench.recorded_traffic("no_such_workload", "block", "radial") is None
+    # a record taken on other sources is not reported
+    fake_root = tmp_path
+    (fake_root / "profiles").mkdir()
+    (fake_root / "profiles" / "attn_fwd_traffic.txt").write_text(
+        "hunyuan108k/radial/block sources=0000000000000000 dram_bytes_per_launch=123\n")
+    for rel in bench.ATTN_SOURCES["fwd"]:
+        dst = fake_root / rel
+        dst.parent.mkdir(parents=True, exist_ok=True)
+        dst.write_bytes(open(os.path.join(ROOT, rel), "rb").read())
+    monkeypatch.setattr(bench, "ROOT", str(fake_root))
+    assert bench.recorded_traffic("hunyuan108k", "block", "radial") is None
+    good = bench.sources_sha256("fwd")
+    (fake_root / "profiles" / "attn_fwd_traffic.txt").write_text(
+        f"hunyuan108k/radial/block sources={good} dram_bytes_per_launch=123\n")
+    assert bench.recorded_traffic("hunyuan108k", "block", "radial") == 123
+
+
+def test_workload_description_names_the_mask(bench):
+    import synth
+    c = synth.CONFIGS["hunyuan108k"]
+    text = bench.workload_desc("hunyuan108k", c["masks"][2], "block", c)
+    assert "3600 global (sink) tokens" in text and "n=108000" in text
+    w = synth.CONFIGS["wan_radial"]
+    assert "W=16" in bench.workload_desc("wan_radial", w["masks"][1], "block", w)
+
+
+def test_pass_choices(bench, monkeypatch):
+    for argv, want in ([["bench.py"], "fwd"], [["bench.py", "--pass", "bwd"], "bwd"],
+                       [["bench.py", "--pass", "stream", "--workload", "wan_radial", "--mask", "1"], "stream"],
+                       [["bench.py", "--pass", "policy"], "policy"]):
+        monkeypatch.setattr(sys, "argv", argv)
+        args = bench.parse_args()
+        assert args.pass_ == want
+        assert args.steps >= 1 and args.warmup >= 3
