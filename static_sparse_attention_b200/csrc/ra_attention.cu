@@ -314,6 +314,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
         if (lane == 0 && L_row > 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, HALF, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(TILE, D, 0, 1);
+            // Descriptors are built once; each MMA only advances the start address
+            // (the issuing thread shares its sub-partition with softmax warps).
+            const uint64_t q_desc = smem_desc_sw128(sQ, 16, 1024);
+            const uint64_t k_desc = smem_desc_sw128(sK, 16, 1024);
+            const uint64_t v_desc = smem_desc_sw128(sV, L::H_CHUNK_BYTES, 1024);  // V as MN-major B
             bool ok = mbar_wait(bar(B_Q_FULL), 0, wc, SITE_Q_FULL);
             tc_fence_after();
             for (int hh = 0; ok && hh <= n_half; ++hh) {
@@ -324,13 +329,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
                     if (!(ok = mbar_wait(bar(B_K_FULL + ks), (hh / L::KS) & 1, wc, SITE_K_FULL)))
                         break;
                     tc_fence_after();
-                    const uint32_t kbase = sK + ks * L::H_BYTES;
+                    const uint64_t kd = desc_add(k_desc, ks * L::H_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        mma_ss(tmem + s_col_of(hh & 1),
-                               smem_desc_sw128(sQ + (kk >> 2) * L::Q_CHUNK_BYTES + (kk & 3) * 32, 16, 1024),
-                               smem_desc_sw128(kbase + (kk >> 2) * L::H_CHUNK_BYTES + (kk & 3) * 32, 16, 1024),
-                               idesc_s, kk > 0 ? 1u : 0u);
+                        mma_ss(tmem + s_col_of(hh & 1), desc_add(q_desc, (kk >> 2) * L::Q_CHUNK_BYTES + (kk & 3) * 32),
+                               desc_add(kd, (kk >> 2) * L::H_CHUNK_BYTES + (kk & 3) * 32), idesc_s, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(bar(B_S_FULL + (hh & 1)));
                     mma_commit(bar(B_K_EMPTY + ks));
@@ -341,17 +344,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
                         !(ok = mbar_wait(bar(B_V_FULL + vs), (j / L::VS) & 1, wc, SITE_V_FULL)))
                         break;
                     tc_fence_after();
-                    const uint32_t vbase = sV + vs * L::H_BYTES;
+                    const uint64_t vd = desc_add(v_desc, vs * L::H_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < HALF / 16; ++kk)
-                        mma_ts(tmem + O_COL, tmem + s_col_of(buf) + kk * 8,
-                               smem_desc_sw128(vbase + kk * 2048, L::H_CHUNK_BYTES, 1024), idesc_pv,
+                        mma_ts(tmem + O_COL, tmem + s_col_of(buf) + kk * 8, desc_add(vd, kk * 2048), idesc_pv,
                                (j > 0 || kk > 0) ? 1u : 0u);
                     if (SPLIT_P) {
 #pragma unroll
                         for (int kk = 0; kk < HALF / 16; ++kk)
-                            mma_ts(tmem + O_COL, tmem + s_col_of(buf) + HALF / 2 + kk * 8,
-                                   smem_desc_sw128(vbase + kk * 2048, L::H_CHUNK_BYTES, 1024), idesc_pv, 1u);
+                            mma_ts(tmem + O_COL, tmem + s_col_of(buf) + HALF / 2 + kk * 8, desc_add(vd, kk * 2048),
+                                   idesc_pv, 1u);
                     }
                     mma_commit(bar(B_V_EMPTY + vs));
                     mma_commit(bar(B_PV_DONE));

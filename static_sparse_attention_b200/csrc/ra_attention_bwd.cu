@@ -200,25 +200,28 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
         if (lane == 0 && len > 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, TILE, 0, 0);  // A, B K-major, N = 128
             constexpr uint32_t idesc_acc = idesc_bf16_f32(TILE, D, 0, 1);   // A from TMEM, B MN-major
+            // Descriptors are built once; each MMA only advances the start address
+            // (the issuing thread shares its sub-partition with gradient warps).
+            const uint64_t dQd = smem_desc_sw128(sQ, 16, 1024), dOd = smem_desc_sw128(sDO, 16, 1024);
+            const uint64_t dKd = smem_desc_sw128(sK, 16, 1024), dVd = smem_desc_sw128(sV, 16, 1024);
+            const uint64_t dKmn = smem_desc_sw128(sK, L::CHUNK_BYTES, 1024);  // K tiles as MN-major B
             // D[col] = A(resident 128 x d) * B(128-row tile)^T over d.
-            auto mma_s = [&](uint32_t col, uint32_t a, uint32_t b2) {
+            auto mma_s = [&](uint32_t col, uint64_t a, uint64_t b2) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
-                    mma_ss(tmem + col, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b2 + off, 16, 1024),
-                           idesc_s, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + col, desc_add(a, off), desc_add(b2, off), idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             // dQ += dS_j K_j: dS packed by the warpgroups, keys 16 kk .. 16 kk + 15
             // at columns 64 (kk / 4) + 8 (kk % 4) of the step's S buffer.
             auto issue_acc = [&](int j) {
                 const int bf = j & 1, ks = j % L::KS;
-                const uint32_t kbase = sK + ks * L::TILE_BYTES;
+                const uint64_t kdesc = desc_add(dKmn, ks * L::TILE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < TILE / 16; ++kk)
                     mma_ts(tmem + DQ_COL_ACC, tmem + dq_s_col(bf) + (kk >> 2) * 64 + (kk & 3) * 8,
-                           smem_desc_sw128(kbase + kk * 2048, L::CHUNK_BYTES, 1024), idesc_acc,
-                           (j > 0 || kk > 0) ? 1u : 0u);
+                           desc_add(kdesc, kk * 2048), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(bar(BB::ACC_DONE + bf));
                 mma_commit(bar(BB::K_EMPTY + ks));
             };
@@ -233,7 +236,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
                 if (j >= 1 && !(ok = mbar_wait(bar(BB::DP_FREE), (j - 1) & 1, wc, BSITE_DS_FULL)))
                     break;
                 tc_fence_after();
-                mma_s(DQ_COL_DP, sDO, sV + vs * L::TILE_BYTES);
+                mma_s(DQ_COL_DP, dOd, desc_add(dVd, vs * L::TILE_BYTES));
                 mma_commit(bar(BB::V_EMPTY + vs));
                 // S_j into buffer bf, once the gradient MMA of step j - 2 (which read
                 // dS from that buffer) has completed: MMAs into different
@@ -243,7 +246,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
                 if (j >= 2 && !(ok = mbar_wait(bar(BB::ACC_DONE + bf), ((j - 2) >> 1) & 1, wc, BSITE_ACC)))
                     break;
                 tc_fence_after();
-                mma_s(dq_s_col(bf), sQ, sK + ks * L::TILE_BYTES);
+                mma_s(dq_s_col(bf), dQd, desc_add(dKd, ks * L::TILE_BYTES));
                 mma_commit(bar(BB::S_FULL + bf));
                 if (j >= 1) {
                     if (!(ok = mbar_wait(bar(BB::DS_FULL + (bf ^ 1)), ((j - 1) >> 1) & 1, wc, BSITE_DS_FULL)))
@@ -520,37 +523,41 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
         if (lane == 0 && len > 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, TILE, 0, 0);  // A, B K-major, N = 128
             constexpr uint32_t idesc_acc = idesc_bf16_f32(TILE, D, 0, 1);   // A K-major, B MN-major
+            // Descriptors are built once; each MMA only advances the start address
+            // (the issuing thread shares its sub-partition with gradient warps).
+            const uint64_t dKd = smem_desc_sw128(sK, 16, 1024), dVd = smem_desc_sw128(sV, 16, 1024);
+            const uint64_t dQd = smem_desc_sw128(sQ, 16, 1024), dOd = smem_desc_sw128(sO, 16, 1024);
+            const uint64_t dPTd = smem_desc_sw128(sPT, 16, 1024);
+            const uint64_t dQmn = smem_desc_sw128(sQ, L::CHUNK_BYTES, 1024);  // Q tiles as MN-major B
+            const uint64_t dOmn = smem_desc_sw128(sO, L::CHUNK_BYTES, 1024);  // dO tiles as MN-major B
             // D[col] = A(resident 128 x d) * B(128-row tile)^T over d.
-            auto mma_s = [&](uint32_t col, uint32_t a, uint32_t b2) {
+            auto mma_s = [&](uint32_t col, uint64_t a, uint64_t b2) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
-                    mma_ss(tmem + col, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b2 + off, 16, 1024),
-                           idesc_s, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + col, desc_add(a, off), desc_add(b2, off), idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             // dK += dS^T_j Q_j: dS^T packed by the warpgroups, queries 16 kk .. 16 kk + 15
             // at columns 64 (kk / 4) + 8 (kk % 4) of the dP^T buffer.
             auto issue_dk = [&](int j) {
                 const int qs = j % L::QS;
-                const uint32_t qbase = sQ + qs * L::TILE_BYTES;
+                const uint64_t qdesc = desc_add(dQmn, qs * L::TILE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < TILE / 16; ++kk)
                     mma_ts(tmem + KV_COL_DK, tmem + KV_COL_DP + (kk >> 2) * 64 + (kk & 3) * 8,
-                           smem_desc_sw128(qbase + kk * 2048, L::CHUNK_BYTES, 1024), idesc_acc,
-                           (j > 0 || kk > 0) ? 1u : 0u);
+                           desc_add(qdesc, kk * 2048), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(bar(BB::DK_DONE));
                 mma_commit(bar(BB::Q_EMPTY + qs));
             };
             // dV += P^T_j dO_j: P^T from shared memory (K-major over the queries).
             auto issue_dv = [&](int j) {
                 const int os = j % L::OS;
-                const uint32_t obase = sO + os * L::TILE_BYTES;
+                const uint64_t odesc = desc_add(dOmn, os * L::TILE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < TILE / 16; ++kk)
-                    mma_ss(tmem + KV_COL_DV, smem_desc_sw128(sPT + (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32, 16, 1024),
-                           smem_desc_sw128(obase + kk * 2048, L::CHUNK_BYTES, 1024), idesc_acc,
-                           (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_ss(tmem + KV_COL_DV, desc_add(dPTd, (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32),
+                           desc_add(odesc, kk * 2048), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(bar(BB::DV_DONE));
                 mma_commit(bar(BB::O_EMPTY + os));
             };
@@ -558,12 +565,12 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                       mbar_wait(bar(BB::Q_FULL), 0, wc, BSITE_X_FULL);
             if (ok) {
                 tc_fence_after();
-                mma_s(KV_COL_S, sK, sQ);
+                mma_s(KV_COL_S, dKd, dQd);
                 ok = mbar_wait(bar(BB::O_FULL), 0, wc, BSITE_Y_FULL);
             }
             if (ok) {
                 tc_fence_after();
-                mma_s(KV_COL_DP, sV, sO);
+                mma_s(KV_COL_DP, dVd, dOd);
                 mma_commit(bar(BB::S_FULL));
             }
             for (int j = 0; ok && j < len; ++j) {
@@ -574,7 +581,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                         !(ok = mbar_wait(bar(BB::S_FREE), j & 1, wc, BSITE_S_FULL)))
                         break;
                     tc_fence_after();
-                    mma_s(KV_COL_S, sK, sQ + (jn % L::QS) * L::TILE_BYTES);
+                    mma_s(KV_COL_S, dKd, desc_add(dQd, (jn % L::QS) * L::TILE_BYTES));
                 }
                 if (!(ok = mbar_wait(bar(BB::DS_FULL), j & 1, wc, BSITE_DS_FULL)))
                     break;
@@ -589,7 +596,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                         !(ok = mbar_wait(bar(BB::DK_DONE), j & 1, wc, BSITE_ACC)))
                         break;
                     tc_fence_after();
-                    mma_s(KV_COL_DP, sV, sO + (jn % L::OS) * L::TILE_BYTES);
+                    mma_s(KV_COL_DP, dVd, desc_add(dOd, (jn % L::OS) * L::TILE_BYTES));
                     mma_commit(bar(BB::S_FULL));
                 }
                 issue_dv(j);

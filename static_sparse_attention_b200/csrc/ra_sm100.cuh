@@ -266,6 +266,15 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
+// The descriptor of the matrix off_bytes (a 16-byte multiple) further on.  The
+// start address field holds bits 4-17 of the address in bits 0-13, and shared
+// memory addresses stay below 2^18, so only the low word changes (no carry).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t off_bytes)
+{
+    const uint32_t lo = static_cast<uint32_t>(d) + (off_bytes >> 4);
+    return (d & 0xFFFFFFFF00000000ull) | lo;
+}
+
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, M x N, operand majors.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major, int b_mn_major)
 {
