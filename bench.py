@@ -199,6 +199,29 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def time_two_streams(step, n_steps, main_stream):
+    """End-to-end timing with two CUDA streams: step i (which enqueues its own
+    host-to-device copies, kernels and device-to-host copy on the stream it is
+    given) runs on stream i % 2 with its own staging buffers, so one step's
+    copies overlap another step's kernels.  Returns the device time in ms from
+    before the first step to after the last."""
+    import torch
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main_stream)
+    for st in streams:
+        st.wait_event(e0)
+    for i in range(n_steps):
+        step(i, streams[i % 2])
+    for st in streams:
+        ev = torch.cuda.Event()
+        ev.record(st)
+        main_stream.wait_event(ev)
+    e1.record(main_stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
 def flops_per_call(info, c, mode, kind="fwd"):
     pairs = info["block_pairs"] if mode == "block" else info["kept_pairs"]
     return (4.0 if kind == "fwd" else 10.0) * c["d"] * pairs * c["B"] * c["H"]
@@ -688,61 +711,60 @@ def main():
     # ---- end to end: host buffers through the C ABI (H2D + kernel + D2H per step)
     e2e = None
     if not args.no_e2e and bwd:
-        # pinned host Q, K, V, O, dO, lse -> device, the backward, dQ, dK, dV -> pinned host
+        # per step: pinned host Q, K, V, O, dO, lse -> device, the backward, dQ, dK, dV -> pinned
+        # host; consecutive steps on two streams with their own device buffers
         hosts = [torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).pin_memory() for h in host]
-        hosts.append(torch.from_numpy(host[0].view(np.int16)).view(torch.bfloat16).pin_memory())  # O slot
-        hosts[4].copy_(o.cpu())
+        hosts.append(o.cpu().pin_memory())  # O
         hl = lse.cpu().pin_memory()
-        houts = [torch.empty(shape, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
-        devs = [q, k, v, do, o]
+        houts = [[torch.empty(shape, dtype=torch.bfloat16).pin_memory() for _ in range(3)] for _ in range(2)]
+        sets = [dict(ins=[q, k, v, do, o], lse=lse, outs=[dq, dk, dv], ws=ws)]
+        sets.append(dict(ins=[torch.empty_like(q) for _ in range(5)], lse=torch.empty_like(lse),
+                         outs=[torch.empty_like(q) for _ in range(3)], ws=torch.empty_like(ws)))
 
-        def e2e_step():
-            for hsrc, dst in zip(hosts, devs):
-                dst.copy_(hsrc, non_blocking=True)
-            lse.copy_(hl, non_blocking=True)
-            step()
-            for hdst, src in zip(houts, (dq, dk, dv)):
-                hdst.copy_(src, non_blocking=True)
+        def e2e_step(i, st):
+            b_ = sets[i % 2]
+            with torch.cuda.stream(st):
+                for hsrc, dst in zip(hosts, b_["ins"]):
+                    dst.copy_(hsrc, non_blocking=True)
+                b_["lse"].copy_(hl, non_blocking=True)
+                qi, ki, vi, doi, oi = b_["ins"]
+                ra.attention_bwd(qi, ki, vi, oi, doi, b_["lse"], m, scale=scale, mode=args.mode, dq=b_["outs"][0],
+                                 dk=b_["outs"][1], dv=b_["outs"][2], workspace=b_["ws"], stream=st)
+                for hdst, src in zip(houts[i % 2], b_["outs"]):
+                    hdst.copy_(src, non_blocking=True)
 
-        e2e_steps = max(3, min(args.steps, 10))
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
+        e2e_steps = max(4, min(args.steps, 10))
+        time_two_streams(e2e_step, 2, stream)  # warm-up
         barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
+        e_ms = max_over_ranks(time_two_streams(e2e_step, e2e_steps, stream), world, f"cuda:{dev}")
         barrier()
-        e_ms = max_over_ranks(e0.elapsed_time(e1), world, f"cuda:{dev}")
         e2e = {"value": flop * e2e_steps * world / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e_ms / e2e_steps, "h2d_bytes_per_step": 5 * q.numel() * 2 + lse.numel() * 4,
                "d2h_bytes_per_step": 3 * q.numel() * 2,
-               "path": "pinned host Q,K,V,O,dO,lse -> device, ra_attention_bwd, device -> pinned host dQ,dK,dV"}
-        del hosts, houts, hl
+               "path": "per step: pinned host Q,K,V,O,dO,lse -> device, ra_attention_bwd, device -> pinned host "
+                       "dQ,dK,dV; consecutive steps on two streams with their own device buffers"}
+        del hosts, houts, hl, sets
     if not args.no_e2e and not bwd:
         hq, hk, hv = (torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).pin_memory() for h in host)
-        ho = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
-        e2e_steps = max(3, min(args.steps, 10))
-        for _ in range(2):
-            ra.attention_fwd_host(hq, hk, hv, ho, q, k, v, o, m, scale=scale, mode=args.mode, stream=stream)
-        torch.cuda.synchronize()
+        ho = [torch.empty(shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        dev_sets = [(q, k, v, o), tuple(torch.empty_like(q) for _ in range(4))]  # staging per stream
+        e2e_steps = max(4, min(args.steps, 10))
+
+        def e2e_step(i, st):
+            dq_, dk_, dv_, do_ = dev_sets[i % 2]
+            ra.attention_fwd_host(hq, hk, hv, ho[i % 2], dq_, dk_, dv_, do_, m, scale=scale, mode=args.mode,
+                                  stream=st)
+
+        time_two_streams(e2e_step, 2, stream)  # warm-up
         barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            ra.attention_fwd_host(hq, hk, hv, ho, q, k, v, o, m, scale=scale, mode=args.mode, stream=stream)
-        e1.record(stream)
-        torch.cuda.synchronize()
+        e_ms = max_over_ranks(time_two_streams(e2e_step, e2e_steps, stream), world, f"cuda:{dev}")
         barrier()
-        e_ms = max_over_ranks(e0.elapsed_time(e1), world, f"cuda:{dev}")
         e2e = {"value": flop * e2e_steps * world / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e_ms / e2e_steps, "h2d_bytes_per_step": 3 * q.numel() * 2,
                "d2h_bytes_per_step": o.numel() * 2,
-               "path": "ra_attention_fwd_host (pinned host Q,K,V -> device, kernel, device -> pinned host O)"}
-        del hq, hk, hv, ho
+               "path": "ra_attention_fwd_host per step (pinned host Q,K,V -> device, kernel, device -> pinned "
+                       "host O), consecutive steps on two streams with their own staging buffers"}
+        del hq, hk, hv, ho, dev_sets
 
     # ---- the same kernel with the dense mask on the same inputs (reference point)
     dense_ref = None
