@@ -73,6 +73,81 @@ __device__ __forceinline__ bool sync_and_wg(uint32_t id, bool pred)
     return out != 0;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 instructions): one instruction for two
+// lanes' worth of IEEE fma / add / mul, each rounded to nearest as the scalar
+// forms are, so the gradients keep the same bits as with scalar arithmetic.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2pack_u(uint32_t lo, uint32_t hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// Gradient of one pair of walked columns: p = 2^(s c + nl), ds = p (dp + nd),
+// where nl = -L log2 e and nd = -D of the pair's rows.  A masked-out element
+// arrives as s = -inf (c > 0), so its p is exactly 0.
+__device__ __forceinline__ void grad_pair(uint32_t s0, uint32_t s1, uint32_t dp0, uint32_t dp1, uint64_t c2,
+                                          uint64_t nl2, uint64_t nd2, float& p0, float& p1, float& ds0, float& ds1)
+{
+    float x0, x1;
+    f2unpack(f2fma(f2pack_u(s0, s1), c2, nl2), x0, x1);
+    p0 = fast_exp2(x0);
+    p1 = fast_exp2(x1);
+    f2unpack(f2mul(f2pack(p0, p1), f2add(f2pack_u(dp0, dp1), nd2)), ds0, ds1);
+}
+
+// The same with explicit keep bits: p = 0 where a bit is clear.  The dK / dV
+// walk uses it on every tile (its keep bits are all set outside token-exact
+// partial tiles); the -inf pass of mask_chunk costs that kernel a register
+// spill.
+__device__ __forceinline__ void grad_pair_keep(uint32_t s0, uint32_t s1, uint32_t dp0, uint32_t dp1, uint64_t c2,
+                                               uint64_t nl2, uint64_t nd2, bool k0, bool k1, float& p0, float& p1,
+                                               float& ds0, float& ds1)
+{
+    float x0, x1;
+    f2unpack(f2fma(f2pack_u(s0, s1), c2, nl2), x0, x1);
+    p0 = k0 ? fast_exp2(x0) : 0.f;
+    p1 = k1 ? fast_exp2(x1) : 0.f;
+    f2unpack(f2mul(f2pack(p0, p1), f2add(f2pack_u(dp0, dp1), nd2)), ds0, ds1);
+}
+
+// Sets the elements of a 32-column chunk of S whose bit in `keep` is clear to -inf.
+__device__ __forceinline__ void mask_chunk(uint32_t (&s)[32], uint32_t keep)
+{
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+        if (!((keep >> e) & 1u))
+            s[e] = __float_as_uint(-INFINITY);
+}
+
 // ---------------------------------------------------------------------------
 // dQ kernel with 128-key steps.  A tcgen05.mma of M = 128 runs at the full
 // rate only for N >= 128 (N = 64 reaches about two thirds), so S = Q K^T and
@@ -277,6 +352,9 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
         const bool tail = (n % TILE) != 0;
         const float row_l2 = row_valid ? p.lse[static_cast<size_t>(bh) * n + row] * LOG2E : 0.f;
         const float row_d = row_valid ? p.Dv[static_cast<size_t>(bh) * n + row] : 0.f;
+        // a row with no kept key (lse = -inf) has P = 0 everywhere
+        const float nl = row_l2 > -INFINITY ? -row_l2 : -INFINITY;
+        const uint64_t c2 = f2pack(p.scale_log2, p.scale_log2), nl2 = f2pack(nl, nl), nd2 = f2pack(-row_d, -row_d);
         bool ok = true;
         // CSR entry of the next step, loaded one step ahead of its use
         int next_kb = len > 0 ? p.idx[start] : 0;
@@ -321,19 +399,14 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
             for (int c = 0; c < 2; ++c) {
                 if (c == 1)
                     tmem_wait_ld();
-                const uint32_t mword = wg ? (c ? mk[3] : mk[2]) : (c ? mk[1] : mk[0]);
+                if (masked)  // warp-uniform
+                    mask_chunk(sv[c], wg ? (c ? mk[3] : mk[2]) : (c ? mk[1] : mk[0]));
                 uint32_t dk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    float ds[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const bool keep = !masked || ((mword >> (e + u)) & 1u);
-                        const float x = fmaf(__uint_as_float(sv[c][e + u]), p.scale_log2, -row_l2);
-                        const float pe = keep ? fast_exp2(x) : 0.f;
-                        ds[u] = pe * (__uint_as_float(dv[c][e + u]) - row_d);
-                    }
-                    dk[e >> 1] = pack_bf16(ds[0], ds[1]);
+                    float p0, p1, ds0, ds1;
+                    grad_pair(sv[c][e], sv[c][e + 1], dv[c][e], dv[c][e + 1], c2, nl2, nd2, p0, p1, ds0, ds1);
+                    dk[e >> 1] = pack_bf16(ds0, ds1);
                 }
                 // Packed into columns this warpgroup has already read.
                 tmem_st16(lane_base + dq_s_col(bf) + my_col + c * 16, dk);
@@ -617,16 +690,21 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
         // this thread's row of P^T (K-major, 128-byte swizzle): chunk wg holds its 64 queries
         uint8_t* pt_row = smem + L::PT_OFF + wg * L::CHUNK_BYTES + t * 128;
         bool ok = true;
-        // Statistic of one query column of the step's (this warpgroup's 64):
-        // threads 0-63 the lse in log2 units (+inf beyond n, so P is exactly 0
-        // there), threads 64-127 D.  Loaded one step ahead of its use, with the
+        // Statistic of one query column of the step's (this warpgroup's 64),
+        // negated: threads 0-63 -L log2 e (-inf beyond n, so P is exactly 0
+        // there), threads 64-127 -D.  Loaded one step ahead of its use, with the
         // CSR entry.
         auto column_stat = [&](int qblock) -> float {
             const int q = qblock * TILE + static_cast<int>(my_col) + (t & 63);
             if (q >= n)
-                return t < 64 ? INFINITY : 0.f;
-            return t < 64 ? p.lse[static_cast<size_t>(bh) * n + q] * LOG2E : p.Dv[static_cast<size_t>(bh) * n + q];
+                return t < 64 ? -INFINITY : -0.f;
+            if (t >= 64)
+                return -p.Dv[static_cast<size_t>(bh) * n + q];
+            // a query row with no kept key (lse = -inf) has P = 0 everywhere
+            const float l = p.lse[static_cast<size_t>(bh) * n + q];
+            return l > -INFINITY ? -(l * LOG2E) : -INFINITY;
         };
+        const uint64_t c2 = f2pack(p.scale_log2, p.scale_log2);
         int next_qb = len > 0 ? p.idx[start] : 0;
         int next_flag = len > 0 ? p.flag[start] : 0;
         float next_stat = len > 0 ? column_stat(next_qb) : 0.f;
@@ -639,9 +717,14 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                 next_flag = p.flag[start + j + 1];
                 next_stat = column_stat(next_qb);
             }
-            uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
-            if (masked && row_valid)
-                col_keep_mask(p.g, rf, rp, qb * TILE, mk[0], mk[1], mk[2], mk[3]);
+            // keep bits of this warpgroup's two 32-column chunks
+            uint32_t mk[2] = {~0u, ~0u};
+            if (masked && row_valid) {
+                uint32_t m4[4];
+                col_keep_mask(p.g, rf, rp, qb * TILE, m4[0], m4[1], m4[2], m4[3]);
+                mk[0] = wg ? m4[2] : m4[0];
+                mk[1] = wg ? m4[3] : m4[1];
+            }
             sync_wg(wg_bar);  // the previous step's readers of the statistics are done
             (t < 64 ? st_l2 : st_d)[my_col + (t & 63)] = stat;
             ok = ok && mbar_wait(bar(BB::S_FULL), j & 1, wc, BSITE_S_FULL);
@@ -664,24 +747,19 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
             for (int c = 0; c < 2; ++c) {
                 if (c == 1)
                     tmem_wait_ld();
-                const uint32_t (&dvc)[32] = dv[c];
-                const uint32_t mword = wg ? (c ? mk[3] : mk[2]) : (c ? mk[1] : mk[0]);
                 const float4* l2v = reinterpret_cast<const float4*>(st_l2 + my_col + c * 32);
                 const float4* dsv = reinterpret_cast<const float4*>(st_d + my_col + c * 32);
                 uint32_t pk[16], dk[16];
 #pragma unroll
                 for (int e4 = 0; e4 < 32; e4 += 4) {
                     const float4 l4 = l2v[e4 >> 2], d4 = dsv[e4 >> 2];  // same address in every lane
-                    const float lq[4] = {l4.x, l4.y, l4.z, l4.w}, dq[4] = {d4.x, d4.y, d4.z, d4.w};
                     float pe[4], ds[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int e = e4 + u;
-                        const bool keep = !masked || ((mword >> e) & 1u);
-                        const float x = fmaf(__uint_as_float(sv[c][e]), p.scale_log2, -lq[u]);
-                        pe[u] = keep ? fast_exp2(x) : 0.f;
-                        ds[u] = pe[u] * (__uint_as_float(dvc[e]) - dq[u]);
-                    }
+                    grad_pair_keep(sv[c][e4], sv[c][e4 + 1], dv[c][e4], dv[c][e4 + 1], c2, f2pack(l4.x, l4.y),
+                                   f2pack(d4.x, d4.y), (mk[c] >> e4) & 1u, (mk[c] >> (e4 + 1)) & 1u, pe[0], pe[1],
+                                   ds[0], ds[1]);
+                    grad_pair_keep(sv[c][e4 + 2], sv[c][e4 + 3], dv[c][e4 + 2], dv[c][e4 + 3], c2,
+                                   f2pack(l4.z, l4.w), f2pack(d4.z, d4.w), (mk[c] >> (e4 + 2)) & 1u,
+                                   (mk[c] >> (e4 + 3)) & 1u, pe[2], pe[3], ds[2], ds[3]);
                     pk[e4 >> 1] = pack_bf16(pe[0], pe[1]);
                     pk[(e4 >> 1) + 1] = pack_bf16(pe[2], pe[3]);
                     dk[e4 >> 1] = pack_bf16(ds[0], ds[1]);
