@@ -15,7 +15,8 @@
 //              (bf16) back over S, and at the end runs the epilogue O / l.
 //   warp 4     producer: TMA loads of Q once, then the K and V half-tiles of
 //              the row into two rings (128-byte swizzle).
-//   warp 5     MMA: allocates TMEM; one thread issues S_h = Q K_h^T
+//   warp 5     MMA: allocates TMEM; runs its loop warp-wide (descriptor
+//              arithmetic warp-uniform) and one elected lane issues S_h = Q K_h^T
 //              (tcgen05.mma, N = 64) into S buffer h % 2 and O += P_h V_h
 //              (A = P from TMEM), in the order S_0, S_1, PV_0, S_2, PV_1, ...:
 //              S of the next half-tile is in flight while the softmax works on
@@ -311,56 +312,74 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
         }
     } else if (warp == 5) {
         // ----------------------------------------------------------------- MMA
-        if (lane == 0 && L_row > 0) {
+        // The whole warp runs the loop, so that the descriptors (built once; each
+        // MMA only advances the start address) stay warp-uniform; the elected
+        // lane issues the MMAs and commits.  The warp shares its sub-partition
+        // with softmax warps.
+        if (L_row > 0) {
+            const bool leader = elect_one();
             constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, HALF, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(TILE, D, 0, 1);
-            // Descriptors are built once; each MMA only advances the start address
-            // (the issuing thread shares its sub-partition with softmax warps).
             const uint64_t q_desc = smem_desc_sw128(sQ, 16, 1024);
             const uint64_t k_desc = smem_desc_sw128(sK, 16, 1024);
             const uint64_t v_desc = smem_desc_sw128(sV, L::H_CHUNK_BYTES, 1024);  // V as MN-major B
-            bool ok = mbar_wait(bar(B_Q_FULL), 0, wc, SITE_Q_FULL);
+            auto wait_all = [&](uint32_t b, uint32_t parity, int site) {
+                return __all_sync(0xFFFFFFFFu, mbar_wait(b, parity, wc, site));
+            };
+            bool ok = wait_all(bar(B_Q_FULL), 0, SITE_Q_FULL);
             tc_fence_after();
             for (int hh = 0; ok && hh <= n_half; ++hh) {
                 if (hh < n_half) {
                     // S_hh into buffer hh % 2; its previous occupant's P V
                     // (half-tile hh - 2) was issued in the previous iteration.
                     const int ks = hh % L::KS;
-                    if (!(ok = mbar_wait(bar(B_K_FULL + ks), (hh / L::KS) & 1, wc, SITE_K_FULL)))
+                    if (!(ok = wait_all(bar(B_K_FULL + ks), (hh / L::KS) & 1, SITE_K_FULL)))
                         break;
                     tc_fence_after();
                     const uint64_t kd = desc_add(k_desc, ks * L::H_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        mma_ss(tmem + s_col_of(hh & 1), desc_add(q_desc, (kk >> 2) * L::Q_CHUNK_BYTES + (kk & 3) * 32),
-                               desc_add(kd, (kk >> 2) * L::H_CHUNK_BYTES + (kk & 3) * 32), idesc_s, kk > 0 ? 1u : 0u);
+                        const uint64_t ad = desc_add(q_desc, (kk >> 2) * L::Q_CHUNK_BYTES + (kk & 3) * 32);
+                        const uint64_t bd = desc_add(kd, (kk >> 2) * L::H_CHUNK_BYTES + (kk & 3) * 32);
+                        if (leader)
+                            mma_ss(tmem + s_col_of(hh & 1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                     }
-                    mma_commit(bar(B_S_FULL + (hh & 1)));
-                    mma_commit(bar(B_K_EMPTY + ks));
+                    if (leader) {
+                        mma_commit(bar(B_S_FULL + (hh & 1)));
+                        mma_commit(bar(B_K_EMPTY + ks));
+                    }
                 }
                 if (hh >= 1) {
                     const int j = hh - 1, vs = j % L::VS, buf = j & 1;
-                    if (!(ok = mbar_wait(bar(B_P_FULL + buf), (j >> 1) & 1, wc, SITE_P_FULL)) ||
-                        !(ok = mbar_wait(bar(B_V_FULL + vs), (j / L::VS) & 1, wc, SITE_V_FULL)))
+                    if (!(ok = wait_all(bar(B_P_FULL + buf), (j >> 1) & 1, SITE_P_FULL)) ||
+                        !(ok = wait_all(bar(B_V_FULL + vs), (j / L::VS) & 1, SITE_V_FULL)))
                         break;
                     tc_fence_after();
                     const uint64_t vd = desc_add(v_desc, vs * L::H_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < HALF / 16; ++kk)
-                        mma_ts(tmem + O_COL, tmem + s_col_of(buf) + kk * 8, desc_add(vd, kk * 2048), idesc_pv,
-                               (j > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < HALF / 16; ++kk) {
+                        const uint64_t bd = desc_add(vd, kk * 2048);
+                        if (leader)
+                            mma_ts(tmem + O_COL, tmem + s_col_of(buf) + kk * 8, bd, idesc_pv,
+                                   (j > 0 || kk > 0) ? 1u : 0u);
+                    }
                     if (SPLIT_P) {
 #pragma unroll
-                        for (int kk = 0; kk < HALF / 16; ++kk)
-                            mma_ts(tmem + O_COL, tmem + s_col_of(buf) + HALF / 2 + kk * 8, desc_add(vd, kk * 2048),
-                                   idesc_pv, 1u);
+                        for (int kk = 0; kk < HALF / 16; ++kk) {
+                            const uint64_t bd = desc_add(vd, kk * 2048);
+                            if (leader)
+                                mma_ts(tmem + O_COL, tmem + s_col_of(buf) + HALF / 2 + kk * 8, bd, idesc_pv, 1u);
+                        }
                     }
-                    mma_commit(bar(B_V_EMPTY + vs));
-                    mma_commit(bar(B_PV_DONE));
+                    if (leader) {
+                        mma_commit(bar(B_V_EMPTY + vs));
+                        mma_commit(bar(B_PV_DONE));
+                    }
                 }
             }
-            mma_commit(bar(B_O_FINAL));
-            // Every MMA issued by this thread has completed once O_FINAL fires.
+            if (leader)
+                mma_commit(bar(B_O_FINAL));
+            // Every MMA issued by the elected lane has completed once O_FINAL fires.
             drain_wait(bar(B_O_FINAL), 0, p.timeout_ns);
         }
     } else {

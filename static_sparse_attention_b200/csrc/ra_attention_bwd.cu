@@ -272,11 +272,14 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
         }
     } else if (warp == DQ_MMA_WARP) {
         // ----------------------------------------------------------------- MMA
-        if (lane == 0 && len > 0) {
+        if (len > 0) {
+            const bool leader = elect_one();
             constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, TILE, 0, 0);  // A, B K-major, N = 128
             constexpr uint32_t idesc_acc = idesc_bf16_f32(TILE, D, 0, 1);   // A from TMEM, B MN-major
-            // Descriptors are built once; each MMA only advances the start address
-            // (the issuing thread shares its sub-partition with gradient warps).
+            // The whole warp runs the loop, so that the descriptors (built once;
+            // each MMA only advances the start address) stay warp-uniform; the
+            // elected lane issues the MMAs and commits.  The warp shares its
+            // sub-partition with gradient warps.
             const uint64_t dQd = smem_desc_sw128(sQ, 16, 1024), dOd = smem_desc_sw128(sDO, 16, 1024);
             const uint64_t dKd = smem_desc_sw128(sK, 16, 1024), dVd = smem_desc_sw128(sV, 16, 1024);
             const uint64_t dKmn = smem_desc_sw128(sK, L::CHUNK_BYTES, 1024);  // K tiles as MN-major B
@@ -285,7 +288,9 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
-                    mma_ss(tmem + col, desc_add(a, off), desc_add(b2, off), idesc_s, kk > 0 ? 1u : 0u);
+                    const uint64_t ad = desc_add(a, off), bd = desc_add(b2, off);
+                    if (leader)
+                        mma_ss(tmem + col, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             // dQ += dS_j K_j: dS packed by the warpgroups, keys 16 kk .. 16 kk + 15
@@ -294,37 +299,47 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
                 const int bf = j & 1, ks = j % L::KS;
                 const uint64_t kdesc = desc_add(dKmn, ks * L::TILE_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < TILE / 16; ++kk)
-                    mma_ts(tmem + DQ_COL_ACC, tmem + dq_s_col(bf) + (kk >> 2) * 64 + (kk & 3) * 8,
-                           desc_add(kdesc, kk * 2048), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(bar(BB::ACC_DONE + bf));
-                mma_commit(bar(BB::K_EMPTY + ks));
+                for (int kk = 0; kk < TILE / 16; ++kk) {
+                    const uint64_t bd = desc_add(kdesc, kk * 2048);
+                    if (leader)
+                        mma_ts(tmem + DQ_COL_ACC, tmem + dq_s_col(bf) + (kk >> 2) * 64 + (kk & 3) * 8, bd, idesc_acc,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (leader) {
+                    mma_commit(bar(BB::ACC_DONE + bf));
+                    mma_commit(bar(BB::K_EMPTY + ks));
+                }
             };
-            bool ok = mbar_wait(bar(BB::RES_FULL), 0, wc, BSITE_RES);
+            auto wait_all = [&](uint32_t b, uint32_t parity, int site) {
+                return __all_sync(0xFFFFFFFFu, mbar_wait(b, parity, wc, site));
+            };
+            bool ok = wait_all(bar(BB::RES_FULL), 0, BSITE_RES);
             tc_fence_after();
             int acc_issued = 0;
             for (int j = 0; ok && j < len; ++j) {
                 const int bf = j & 1, ks = j % L::KS, vs = j % L::VS;
                 // dP_j into the single dP buffer, once the gradient warps have loaded dP_{j-1}
-                if (!(ok = mbar_wait(bar(BB::V_FULL + vs), (j / L::VS) & 1, wc, BSITE_Y_FULL)))
+                if (!(ok = wait_all(bar(BB::V_FULL + vs), (j / L::VS) & 1, BSITE_Y_FULL)))
                     break;
-                if (j >= 1 && !(ok = mbar_wait(bar(BB::DP_FREE), (j - 1) & 1, wc, BSITE_DS_FULL)))
+                if (j >= 1 && !(ok = wait_all(bar(BB::DP_FREE), (j - 1) & 1, BSITE_DS_FULL)))
                     break;
                 tc_fence_after();
                 mma_s(DQ_COL_DP, dOd, desc_add(dVd, vs * L::TILE_BYTES));
-                mma_commit(bar(BB::V_EMPTY + vs));
+                if (leader)
+                    mma_commit(bar(BB::V_EMPTY + vs));
                 // S_j into buffer bf, once the gradient MMA of step j - 2 (which read
                 // dS from that buffer) has completed: MMAs into different
                 // accumulators are not ordered
-                if (!(ok = mbar_wait(bar(BB::K_FULL + ks), (j / L::KS) & 1, wc, BSITE_X_FULL)))
+                if (!(ok = wait_all(bar(BB::K_FULL + ks), (j / L::KS) & 1, BSITE_X_FULL)))
                     break;
-                if (j >= 2 && !(ok = mbar_wait(bar(BB::ACC_DONE + bf), ((j - 2) >> 1) & 1, wc, BSITE_ACC)))
+                if (j >= 2 && !(ok = wait_all(bar(BB::ACC_DONE + bf), ((j - 2) >> 1) & 1, BSITE_ACC)))
                     break;
                 tc_fence_after();
                 mma_s(dq_s_col(bf), dQd, desc_add(dKd, ks * L::TILE_BYTES));
-                mma_commit(bar(BB::S_FULL + bf));
+                if (leader)
+                    mma_commit(bar(BB::S_FULL + bf));
                 if (j >= 1) {
-                    if (!(ok = mbar_wait(bar(BB::DS_FULL + (bf ^ 1)), ((j - 1) >> 1) & 1, wc, BSITE_DS_FULL)))
+                    if (!(ok = wait_all(bar(BB::DS_FULL + (bf ^ 1)), ((j - 1) >> 1) & 1, BSITE_DS_FULL)))
                         break;
                     tc_fence_after();
                     issue_acc(j - 1);
@@ -332,12 +347,13 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
                 }
             }
             if (ok && acc_issued == len - 1) {
-                if (mbar_wait(bar(BB::DS_FULL + ((len - 1) & 1)), ((len - 1) >> 1) & 1, wc, BSITE_DS_FULL)) {
+                if (wait_all(bar(BB::DS_FULL + ((len - 1) & 1)), ((len - 1) >> 1) & 1, BSITE_DS_FULL)) {
                     tc_fence_after();
                     issue_acc(len - 1);
                 }
             }
-            mma_commit(bar(BB::FINAL));
+            if (leader)
+                mma_commit(bar(BB::FINAL));
             drain_wait(bar(BB::FINAL), 0, p.timeout_ns);
         }
     } else {
@@ -593,11 +609,14 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
         }
     } else if (warp == KV_MMA_WARP) {
         // ----------------------------------------------------------------- MMA
-        if (lane == 0 && len > 0) {
+        if (len > 0) {
+            const bool leader = elect_one();
             constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, TILE, 0, 0);  // A, B K-major, N = 128
             constexpr uint32_t idesc_acc = idesc_bf16_f32(TILE, D, 0, 1);   // A K-major, B MN-major
-            // Descriptors are built once; each MMA only advances the start address
-            // (the issuing thread shares its sub-partition with gradient warps).
+            // The whole warp runs the loop, so that the descriptors (built once;
+            // each MMA only advances the start address) stay warp-uniform; the
+            // elected lane issues the MMAs and commits.  The warp shares its
+            // sub-partition with gradient warps.
             const uint64_t dKd = smem_desc_sw128(sK, 16, 1024), dVd = smem_desc_sw128(sV, 16, 1024);
             const uint64_t dQd = smem_desc_sw128(sQ, 16, 1024), dOd = smem_desc_sw128(sO, 16, 1024);
             const uint64_t dPTd = smem_desc_sw128(sPT, 16, 1024);
@@ -608,7 +627,9 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
-                    mma_ss(tmem + col, desc_add(a, off), desc_add(b2, off), idesc_s, kk > 0 ? 1u : 0u);
+                    const uint64_t ad = desc_add(a, off), bd = desc_add(b2, off);
+                    if (leader)
+                        mma_ss(tmem + col, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             // dK += dS^T_j Q_j: dS^T packed by the warpgroups, queries 16 kk .. 16 kk + 15
@@ -617,46 +638,59 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                 const int qs = j % L::QS;
                 const uint64_t qdesc = desc_add(dQmn, qs * L::TILE_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < TILE / 16; ++kk)
-                    mma_ts(tmem + KV_COL_DK, tmem + KV_COL_DP + (kk >> 2) * 64 + (kk & 3) * 8,
-                           desc_add(qdesc, kk * 2048), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(bar(BB::DK_DONE));
-                mma_commit(bar(BB::Q_EMPTY + qs));
+                for (int kk = 0; kk < TILE / 16; ++kk) {
+                    const uint64_t bd = desc_add(qdesc, kk * 2048);
+                    if (leader)
+                        mma_ts(tmem + KV_COL_DK, tmem + KV_COL_DP + (kk >> 2) * 64 + (kk & 3) * 8, bd, idesc_acc,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (leader) {
+                    mma_commit(bar(BB::DK_DONE));
+                    mma_commit(bar(BB::Q_EMPTY + qs));
+                }
             };
             // dV += P^T_j dO_j: P^T from shared memory (K-major over the queries).
             auto issue_dv = [&](int j) {
                 const int os = j % L::OS;
                 const uint64_t odesc = desc_add(dOmn, os * L::TILE_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < TILE / 16; ++kk)
-                    mma_ss(tmem + KV_COL_DV, desc_add(dPTd, (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32),
-                           desc_add(odesc, kk * 2048), idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(bar(BB::DV_DONE));
-                mma_commit(bar(BB::O_EMPTY + os));
+                for (int kk = 0; kk < TILE / 16; ++kk) {
+                    const uint64_t ad = desc_add(dPTd, (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32);
+                    const uint64_t bd = desc_add(odesc, kk * 2048);
+                    if (leader)
+                        mma_ss(tmem + KV_COL_DV, ad, bd, idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (leader) {
+                    mma_commit(bar(BB::DV_DONE));
+                    mma_commit(bar(BB::O_EMPTY + os));
+                }
             };
-            bool ok = mbar_wait(bar(BB::RES_FULL), 0, wc, BSITE_RES) &&
-                      mbar_wait(bar(BB::Q_FULL), 0, wc, BSITE_X_FULL);
+            auto wait_all = [&](uint32_t b, uint32_t parity, int site) {
+                return __all_sync(0xFFFFFFFFu, mbar_wait(b, parity, wc, site));
+            };
+            bool ok = wait_all(bar(BB::RES_FULL), 0, BSITE_RES) && wait_all(bar(BB::Q_FULL), 0, BSITE_X_FULL);
             if (ok) {
                 tc_fence_after();
                 mma_s(KV_COL_S, dKd, dQd);
-                ok = mbar_wait(bar(BB::O_FULL), 0, wc, BSITE_Y_FULL);
+                ok = wait_all(bar(BB::O_FULL), 0, BSITE_Y_FULL);
             }
             if (ok) {
                 tc_fence_after();
                 mma_s(KV_COL_DP, dVd, dOd);
-                mma_commit(bar(BB::S_FULL));
+                if (leader)
+                    mma_commit(bar(BB::S_FULL));
             }
             for (int j = 0; ok && j < len; ++j) {
                 const int jn = j + 1;
                 if (jn < len) {
                     // S^T_{j+1} over S^T_j, which the gradient warps have loaded
-                    if (!(ok = mbar_wait(bar(BB::Q_FULL + jn % L::QS), (jn / L::QS) & 1, wc, BSITE_X_FULL)) ||
-                        !(ok = mbar_wait(bar(BB::S_FREE), j & 1, wc, BSITE_S_FULL)))
+                    if (!(ok = wait_all(bar(BB::Q_FULL + jn % L::QS), (jn / L::QS) & 1, BSITE_X_FULL)) ||
+                        !(ok = wait_all(bar(BB::S_FREE), j & 1, BSITE_S_FULL)))
                         break;
                     tc_fence_after();
                     mma_s(KV_COL_S, dKd, desc_add(dQd, (jn % L::QS) * L::TILE_BYTES));
                 }
-                if (!(ok = mbar_wait(bar(BB::DS_FULL), j & 1, wc, BSITE_DS_FULL)))
+                if (!(ok = wait_all(bar(BB::DS_FULL), j & 1, BSITE_DS_FULL)))
                     break;
                 tc_fence_after();
                 issue_dk(j);
@@ -665,16 +699,18 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                     // completed (MMAs into different accumulators are not
                     // ordered), and ahead of dV_j, so that the next step's
                     // gradient warps start sooner
-                    if (!(ok = mbar_wait(bar(BB::O_FULL + jn % L::OS), (jn / L::OS) & 1, wc, BSITE_Y_FULL)) ||
-                        !(ok = mbar_wait(bar(BB::DK_DONE), j & 1, wc, BSITE_ACC)))
+                    if (!(ok = wait_all(bar(BB::O_FULL + jn % L::OS), (jn / L::OS) & 1, BSITE_Y_FULL)) ||
+                        !(ok = wait_all(bar(BB::DK_DONE), j & 1, BSITE_ACC)))
                         break;
                     tc_fence_after();
                     mma_s(KV_COL_DP, dVd, desc_add(dOd, (jn % L::OS) * L::TILE_BYTES));
-                    mma_commit(bar(BB::S_FULL));
+                    if (leader)
+                        mma_commit(bar(BB::S_FULL));
                 }
                 issue_dv(j);
             }
-            mma_commit(bar(BB::FINAL));
+            if (leader)
+                mma_commit(bar(BB::FINAL));
             drain_wait(bar(BB::FINAL), 0, p.timeout_ns);
         }
     } else {

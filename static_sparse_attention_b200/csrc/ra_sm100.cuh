@@ -165,6 +165,21 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
         : "memory");
 }
 
+// One lane of the (fully active) warp, the same one on every call.  The MMA
+// warps run their loops warp-wide, so that the descriptor arithmetic stays
+// warp-uniform, and only this lane issues the tcgen05 MMAs and commits (a
+// commit tracks the MMAs of the thread that executes it).
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t is_leader;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(is_leader));
+    return is_leader != 0;
+}
+
 // D[tmem] (+)= A[tmem] * B[smem], kind::f16; A is M x K, K-major, in TMEM.
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate)
