@@ -725,7 +725,7 @@ def main():
                 "peak_source": f"{peak_src} bf16 {'burst' if timed_alone else 'sustained'} (MEASURED_PEAKS.json)"
                 if peak_src == "measured" else "fallback 1.59 PFLOP/s burst / 1.4 sustained",
                 "kernel": ("attn_fwd_kernel<%d>" % d) if not bwd else
-                ("ra_attention_bwd call: bwd_dot_kernel<%d> + bwd_kernel<%d, dQ> + bwd_kernel<%d, dK dV>" % (d, d, d)),
+                ("ra_attention_bwd call: bwd_dot_kernel<%d> + bwd_dq_kernel<%d> + bwd_dkdv_kernel<%d>" % (d, d, d)),
                 "flop_per_launch": flop,
                 "flop_executed_per_launch": flops_per_call(info, c, "block", args.pass_),
                 "algorithmic_bytes_per_launch": bytes_qkvo}
