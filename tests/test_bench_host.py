@@ -69,3 +69,32 @@ def test_pass_choices(bench, monkeypatch):
         args = bench.parse_args()
         assert args.pass_ == want
         assert args.steps >= 1 and args.warmup >= 3
+
+
+def _reference_line(args, rank="0"):
+    import json
+    import subprocess
+    env = dict(os.environ, RANK=rank)
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", *args], cwd=ROOT, env=env,
+                         capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = out.stdout.strip().splitlines()
+    return json.loads(lines[-1]) if lines else None
+
+
+@pytest.mark.parametrize("args", [["--workload", "tiny_radial", "--steps", "1", "--warmup", "3"],
+                                  ["--pass", "stream", "--workload", "wan_radial", "--mask", "1",
+                                   "--steps", "1", "--warmup", "3"]], ids=["fwd_tiny", "stream_wan"])
+def test_reference_arm_line(args):
+    """The reference arm (the oracle on the host cores) prints one line with the
+    contract's keys; a rank other than 0 prints nothing and exits 0."""
+    line = _reference_line(args)
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "TFLOP/s"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert _reference_line(args, rank="1") is None
