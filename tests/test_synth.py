@@ -96,3 +96,21 @@ def test_moments_and_independent_streams():
         assert abs(((x - x.mean()) ** 4).mean() / x.var() ** 2 - 3.0) < 0.05   # normal kurtosis
     for a, b in ((q, k), (q, q2), (k, q2)):
         assert abs(np.corrcoef(a, b)[0, 1]) < bound
+
+
+@pytest.mark.parametrize("f,s", [(30, 3600), (41, 1560), (128, 3600), (1, 100), (3, 40)])
+def test_sampled_rows_hold_the_boundary_rows(f, s):
+    """The seeded rows the full-size parity tests check: distinct, sorted, in range,
+    the requested count, the same for the same seed, and always including the
+    boundary rows (sequence ends, frame 1's first and last row, the last frame's
+    first row, the first row of the ragged last tile)."""
+    n = f * s
+    rows = synth.sample_rows(1234, f, s)
+    assert rows.dtype == np.int64 and len(rows) == min(256, n)
+    assert np.all(np.diff(rows) > 0) and rows[0] >= 0 and rows[-1] < n
+    need = {0, n - 1, (f - 1) * s, ((n + 127) // 128 - 1) * 128}
+    if f > 1:
+        need |= {s, 2 * s - 1}
+    assert need <= set(rows.tolist())
+    np.testing.assert_array_equal(rows, synth.sample_rows(1234, f, s))
+    assert not np.array_equal(rows, synth.sample_rows(1235, f, s)) or n <= 256
