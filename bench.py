@@ -7,15 +7,21 @@ One step = one ra_attention_fwd call over every batch element and head of the
 workload (mask built once beforehand: it is static).  With --pass bwd a step is
 one ra_attention_bwd call instead (dQ, dK, dV from the forward's O and lse and a
 seeded dO), counted at 10 * d FLOP per computed pair per head (the five
-products S, dP, dQ, dK, dV; the kernels recompute S and dP in both passes).  Default workload: the
-HunyuanVideo-shaped radial configuration (f=30 frames, s=3600 tokens per
-frame, n=108000, 24 heads, d=128), eq. 4 mask at 128x128 tiles, block mode.
+products S, dP, dQ, dK, dV; the kernels recompute S and dP in both passes).
+
+Default workload: the largest radial configuration that the metric is quoted
+on, 4x-long (f=128 frames, s=3600 tokens per frame, n=460800, 24 heads, d=128),
+eq. 4 mask at 128x128 tiles, block mode; --workload hunyuan108k gives the
+HunyuanVideo-shaped one (f=30, n=108000).
 
 Throughput is effective TFLOP/s on kept-pair FLOPs: 4 * d per computed
 (query, key) pair per head (2d for Q K^T, 2d for P V); in block mode the
-computed pairs are the valid pairs of the kept tiles.  Under torchrun each rank
-runs the same workload on its own GPU (its own batch element of a global batch
-of N, weak scaling, no collective on the data path); rank 0 prints one JSON line.
+computed pairs are the valid pairs of the kept tiles.  Under torchrun the ranks
+split the heads of the one problem (each rank builds the static mask itself and
+computes its head range; no collective on the data path; strong scaling), or
+with --split batch each rank runs its own batch element (weak scaling); the
+only collective is the max over ranks of the device time.  Rank 0 prints one
+JSON line.
 """
 from __future__ import annotations
 
@@ -55,13 +61,16 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="hunyuan108k", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--workload", default="long460k", choices=sorted(synth.CONFIGS))
     ap.add_argument("--mask", type=int, default=0, help="index into the workload's mask list")
     ap.add_argument("--mode", default="block", choices=["block", "token_exact"])
     ap.add_argument("--no-dense-ref", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (small profiling cases)")
+    ap.add_argument("--split", default="heads", choices=["heads", "batch"],
+                    help="with N > 1 GPUs: split the heads of the one problem over the ranks (strong scaling, "
+                         "default) or give each rank its own batch element (weak scaling)")
     ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd", "stream", "policy"],
                     help="time the forward (default), the backward, the streaming SWC step, or a whole "
                          "dense-first denoising schedule of forward calls")
@@ -184,8 +193,36 @@ def physical_gpu(dev: int) -> str:
 
 
 def rank_tensor_ids(rank: int):
-    """Input streams (Q, K, V) of one rank: its own batch element of the global batch."""
+    """Input streams (Q, K, V) of one rank under the batch split: its own batch
+    element of the global batch."""
     return (3 * rank, 3 * rank + 1, 3 * rank + 2)
+
+
+def head_range(rank: int, world: int, H: int):
+    """Heads [h0, h1) of one problem that rank `rank` of `world` computes under the
+    head split: contiguous ranges, sizes differing by at most one, covering
+    [0, H) exactly once (heads are independent given the shared static mask)."""
+    if not 0 <= rank < world or world > H:
+        raise ValueError(f"cannot split {H} heads over {world} ranks (rank {rank})")
+    base, extra = divmod(H, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
+
+
+def rank_inputs(name: str, c: dict, rank: int, world: int, split: str, extra_ids=()):
+    """This rank's Q, K, V (and any extra tensor ids) as bf16 bit patterns.
+    split == "heads": heads head_range(rank) of the one problem (the same
+    tensors on every rank, sliced); split == "batch": the rank's own batch
+    element (its own input streams)."""
+    B, H, d = c["B"], c["H"], c["d"]
+    n = c["f"] * c["s"]
+    seed = synth.config_seed(name)
+    if split == "heads":
+        h0, h1 = head_range(rank, world, H)
+        ids = (0, 1, 2) + tuple(extra_ids)
+        return [synth.normal_bf16_heads(seed, tid, (B, H, n, d), h0, h1) for tid in ids]
+    ids = rank_tensor_ids(rank) + tuple(t + rank for t in extra_ids)
+    return [synth.normal_bf16(seed, tid, (B, H, n, d)) for tid in ids]
 
 
 def max_over_ranks(value: float, world: int, device=None) -> float:
@@ -642,13 +679,19 @@ def main():
         run_policy(args, c, mask, world, rank, dev)
         return
 
-    B, H, d = c["B"], c["H"], c["d"]
+    bwd = args.pass_ == "bwd"
+    split = args.split if world > 1 else "heads"
+    # This rank's share of the work: a head range of the one problem (head
+    # split), or its own batch element (batch split).  The mask is built
+    # locally on every rank: it is static and shared by all heads.
+    h0, h1 = head_range(rank, world, c["H"]) if split == "heads" else (0, c["H"])
+    c_rank = dict(c, H=h1 - h0)
+    B, H, d = c_rank["B"], c_rank["H"], c_rank["d"]
     n = c["f"] * c["s"]
     shape = (B, H, n, d)
     seed = synth.config_seed(args.workload)
-    # This rank's batch element of the global batch: its own input streams.
-    host = [synth.normal_bf16(seed, tid, shape) for tid in rank_tensor_ids(rank)]
-    q, k, v = (torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).to(f"cuda:{dev}") for h in host)
+    host = rank_inputs(args.workload, c, rank, world, split, (synth.DOUT_TENSOR_ID,) if bwd else ())
+    q, k, v = (torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).to(f"cuda:{dev}") for h in host[:3])
     o = torch.empty_like(q)
     m = ra.build_mask(mask, c["f"], c["s"], c["grid"])
     info = m.info
@@ -656,8 +699,10 @@ def main():
     t_mb = time.perf_counter()
     ra.build_mask(mask, c["f"], c["s"], c["grid"]).free()  # synchronises
     mask_build_ms = (time.perf_counter() - t_mb) * 1e3
-    bwd = args.pass_ == "bwd"
-    flop = flops_per_call(info, c, args.mode, args.pass_)
+    flop = flops_per_call(info, c_rank, args.mode, args.pass_)
+    # FLOP of one step of the whole job: the one problem (head split) or one
+    # problem per rank (batch split)
+    flop_job = flops_per_call(info, c, args.mode, args.pass_) * (1 if split == "heads" else world)
     scale = 1.0 / math.sqrt(d)
     stream = torch.cuda.current_stream()
     bytes_qkvo = 4 * q.numel() * 2
@@ -665,7 +710,6 @@ def main():
 
     if bwd:
         # the backward's inputs: this rank's seeded dO, and O and lse from the forward
-        host.append(synth.normal_bf16(seed, synth.DOUT_TENSOR_ID + rank, shape))
         do = torch.from_numpy(host[3].view(np.int16)).view(torch.bfloat16).to(f"cuda:{dev}")
         lse = torch.empty((B, H, n), dtype=torch.float32, device=f"cuda:{dev}")
         ra.attention_fwd(q, k, v, m, scale=scale, mode=args.mode, out=o, lse=lse, stream=stream)
@@ -712,7 +756,7 @@ def main():
         raise SystemExit(f"device status {status} after the timed region")
     total_ms = max_over_ranks(total_ms, world, f"cuda:{dev}")
     ms_per_step = total_ms / args.steps
-    value = flop * args.steps * world / (total_ms / 1e3) / 1e12
+    value = flop_job * args.steps / (total_ms / 1e3) / 1e12
     avg_launch_s = float(np.mean(launch_ms)) / 1e3
     achieved = flop / avg_launch_s / 1e12
 
@@ -727,7 +771,7 @@ def main():
                 "kernel": ("attn_fwd_kernel<%d>" % d) if not bwd else
                 ("ra_attention_bwd call: bwd_dot_kernel<%d> + bwd_dq_kernel<%d> + bwd_dkdv_kernel<%d>" % (d, d, d)),
                 "flop_per_launch": flop,
-                "flop_executed_per_launch": flops_per_call(info, c, "block", args.pass_),
+                "flop_executed_per_launch": flops_per_call(info, c_rank, "block", args.pass_),
                 "algorithmic_bytes_per_launch": bytes_qkvo}
 
     # ---- end to end: host buffers through the C ABI (H2D + kernel + D2H per step)
@@ -760,7 +804,7 @@ def main():
         barrier()
         e_ms = max_over_ranks(time_two_streams(e2e_step, e2e_steps, stream), world, f"cuda:{dev}")
         barrier()
-        e2e = {"value": flop * e2e_steps * world / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": flop_job * e2e_steps / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e_ms / e2e_steps, "h2d_bytes_per_step": 5 * q.numel() * 2 + lse.numel() * 4,
                "d2h_bytes_per_step": 3 * q.numel() * 2,
                "path": "per step: pinned host Q,K,V,O,dO,lse -> device, ra_attention_bwd, device -> pinned host "
@@ -781,7 +825,7 @@ def main():
         barrier()
         e_ms = max_over_ranks(time_two_streams(e2e_step, e2e_steps, stream), world, f"cuda:{dev}")
         barrier()
-        e2e = {"value": flop * e2e_steps * world / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": flop_job * e2e_steps / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e_ms / e2e_steps, "h2d_bytes_per_step": 3 * q.numel() * 2,
                "d2h_bytes_per_step": o.numel() * 2,
                "path": "ra_attention_fwd_host per step (pinned host Q,K,V -> device, kernel, device -> pinned "
@@ -792,7 +836,7 @@ def main():
     dense_ref = None
     if not args.no_dense_ref and mask["family"] != "dense" and not bwd:
         md = ra.build_mask(dict(family="dense"), c["f"], c["s"])
-        dflop = flops_per_call(md.info, c, "block")
+        dflop = flops_per_call(md.info, c_rank, "block")
         for _ in range(2):
             ra.attention_fwd(q, k, v, md, scale=scale, mode="block", out=o, stream=stream)
         d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -822,13 +866,18 @@ def main():
     line = {
         "metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "strong" if split == "heads" else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {
             "workload": workload_desc(args.workload, mask, args.mode, c),
-            "mask": mask["family"], "mode": args.mode, "pass": args.pass_, "global_batch": B * world, "heads": H,
-            "seq_len": n,
-            "head_dim": d, "parallelism": f"{world} independent problems (one per GPU), no collective",
+            "mask": mask["family"], "mode": args.mode, "pass": args.pass_,
+            "global_batch": c["B"] * (world if split == "batch" else 1), "heads": c["H"], "seq_len": n,
+            "head_dim": d,
+            "parallelism": (f"heads split over {world} GPUs ({H} or fewer heads each, mask built on every rank), "
+                            f"no collective on the data path" if split == "heads" and world > 1 else
+                            f"{world} independent problems (one per GPU), no collective" if world > 1 else
+                            "one GPU"),
             "l2": f"inputs larger than L2: {'Q+K+V+O' if not bwd else 'Q+K+V+O+dO+dQ+dK+dV'} = "
                   f"{bytes_qkvo / 1e9:.2f} GB per GPU vs 126 MB L2",
             "kept_tiles": info["nnz"], "tile_sparsity": 1.0 - info["nnz"] / tile_total,

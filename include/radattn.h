@@ -35,7 +35,11 @@
  *     (NULL = the legacy default stream) and is asynchronous unless stated.
  *   - A kernel that gives up a bounded internal wait records
  *     RA_ERR_DEVICE_TIMEOUT in a per-device error word; ra_get_device_status
- *     reads (and clears) it.  Kernels never trap.
+ *     reads (and clears) it.  Kernels never trap.  The word is sticky: while it
+ *     is set, every later forward, backward or SWC-step kernel on that device
+ *     does no work and leaves its outputs unwritten, although its entry point
+ *     returned RA_OK when it was enqueued.  Check ra_get_device_status before
+ *     trusting outputs produced after a possible timeout; it clears the word.
  *   - Results are deterministic: the same inputs give the same bits.
  */
 #ifndef RADATTN_H
@@ -69,7 +73,8 @@ typedef enum {
     RA_ERR_UNSUPPORTED = 2,
     RA_ERR_CUDA = 3,
     RA_ERR_OUT_OF_MEMORY = 4,
-    RA_ERR_DEVICE_TIMEOUT = 5
+    RA_ERR_DEVICE_TIMEOUT = 5,
+    RA_ERR_DEVICE_BOUNDS = 6 /* debug build only: a kernel's bounds check failed */
 } ra_status;
 
 #define RA_TILE 128 /* tile edge, "Radial Attention" sec. 6 */
@@ -136,9 +141,10 @@ ra_status ra_build_mask(int family, int f, int s, const ra_mask_params* params, 
  *                           is too small (so the caller can size the arrays).
  * Limit: n <= 131072 tokens (nb <= 1024); larger masks get RA_ERR_UNSUPPORTED.
  * RA_ERR_INVALID_ARG if nnz exceeds nnz_capacity (nothing but row_ptr written).
- * Synchronises `stream` once (to read nnz).  The first call on a device looks up
- * the scratch's device address and may load the library's module on that
- * device: make it before any stream capture.  All calls share the one scratch
+ * Every call synchronises `stream` (to read nnz), so no call may be made while
+ * `stream` is being captured into a CUDA graph.  Each call looks up the
+ * scratch's device address in the current context (the first call on a device
+ * may load the library's module there).  All calls share the one scratch
  * array, so calls that can overlap on the GPU (different streams, no ordering)
  * race; calls ordered on one stream are safe.
  */
@@ -206,8 +212,10 @@ ra_status ra_attention_fwd_host(const void* Q_host, const void* K_host, const vo
  *   Q, K, V, O, dO : device, bf16 [B, H, n, d], contiguous, 16-byte aligned;
  *                    O is the forward's output for the same Q, K, V, m, mode.
  *   lse            : device fp32 [B, H, n], the forward's log-sum-exp.
- *   dQ, dK, dV     : device, bf16 [B, H, n, d], written (no aliasing with the inputs).
+ *   dQ, dK, dV     : device, bf16 [B, H, n, d], written.
  *   D_workspace    : device fp32 [B, H, n], caller-owned scratch (receives D).
+ *                    None of dQ, dK, dV, D_workspace may overlap any other
+ *                    buffer of the call (RA_ERR_INVALID_ARG).
  *   d, m, scale, mode : as for ra_attention_fwd (same values as the forward).
  * dQ walks the block-CSR rows, dK and dV the transposed block-CSR; no atomics,
  * so the result is deterministic.  Asynchronous on `stream`; no allocation.
@@ -262,6 +270,16 @@ ra_status ra_get_device_error_site(int* site, int* block);
  * it observed, RA_ERR_DEVICE_TIMEOUT when the bound works; the error word is
  * cleared afterwards.  Synchronous. */
 ra_status ra_selftest_wait_timeout(long long timeout_ns, ra_stream stream);
+
+/* Bounds-check self-test.  The library built with -DRA_DEBUG_BOUNDS
+ * (libradattn_debug.so: every global index and TMA coordinate a kernel derives
+ * from its inputs is checked before use, and a failure records
+ * RA_ERR_DEVICE_BOUNDS with its site in the error word and skips the access,
+ * without trapping) launches one CTA whose check fails on an index it never
+ * uses, and returns the device status it observed: RA_ERR_DEVICE_BOUNDS when
+ * the checks are compiled in; the error word is cleared afterwards.  The
+ * release library returns RA_ERR_UNSUPPORTED.  Synchronous. */
+ra_status ra_selftest_bounds(ra_stream stream);
 
 /* Limit of every bounded wait in the library's kernels (default 4e9 ns). */
 ra_status ra_set_wait_timeout_ns(long long timeout_ns);

@@ -17,10 +17,16 @@ import math
 import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libradattn.so")
+# RA_LIBRARY_VARIANT=debug selects the build with device-side bounds checks
+# (libradattn_debug.so, `build.py --debug`); the default is the release build.
+VARIANT = os.environ.get("RA_LIBRARY_VARIANT", "release")
+if VARIANT not in ("release", "debug"):
+    raise ImportError(f"RA_LIBRARY_VARIANT must be 'release' or 'debug', not {VARIANT!r}")
+LIB_PATH = os.path.join(_PKG, "libradattn_debug.so" if VARIANT == "debug" else "libradattn.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libradattn.so is not built ({LIB_PATH}); run `python static_sparse_attention_b200/build.py`")
+    raise ImportError(f"{os.path.basename(LIB_PATH)} is not built ({LIB_PATH}); run "
+                      f"`python static_sparse_attention_b200/build.py{' --debug' if VARIANT == 'debug' else ''}`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -28,7 +34,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 RA_MASK_DENSE, RA_MASK_RADIAL, RA_MASK_WINDOW3D, RA_MASK_SWC = 0, 1, 2, 3
 RA_MODE_TOKEN_EXACT, RA_MODE_BLOCK = 0, 1
 RA_TILE_PARTIAL, RA_TILE_FULL = 0, 1
-RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_OUT_OF_MEMORY, RA_ERR_DEVICE_TIMEOUT = range(6)
+(RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_OUT_OF_MEMORY, RA_ERR_DEVICE_TIMEOUT,
+ RA_ERR_DEVICE_BOUNDS) = range(7)
 RA_TILE = 128
 RA_PV_AUTO, RA_PV_BF16, RA_PV_SPLIT = 0, 1, 2
 FAMILIES = {"dense": RA_MASK_DENSE, "radial": RA_MASK_RADIAL, "window3d": RA_MASK_WINDOW3D, "swc": RA_MASK_SWC}
@@ -71,6 +78,7 @@ _SIGS = {
     "ra_get_device_status": ([_vp], _i),
     "ra_get_device_error_site": ([ctypes.POINTER(_i), ctypes.POINTER(_i)], _i),
     "ra_selftest_wait_timeout": ([_ll, _vp], _i),
+    "ra_selftest_bounds": ([_vp], _i),
     "ra_set_wait_timeout_ns": ([_ll], _i),
     "ra_set_pv_precision": ([_i], _i),
     "ra_status_string": ([_i], ctypes.c_char_p),

@@ -100,6 +100,8 @@ extern "C" const char* ra_status_string(ra_status s)
         return "out of device memory";
     case RA_ERR_DEVICE_TIMEOUT:
         return "device wait timed out";
+    case RA_ERR_DEVICE_BOUNDS:
+        return "device bounds check failed";
     }
     return "unknown status";
 }

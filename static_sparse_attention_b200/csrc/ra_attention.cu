@@ -24,10 +24,22 @@
 // TMEM columns: S buffers at 0 and 64 (fp32, 64 columns; P overlays each as
 // packed bf16), O at 128 (fp32, d columns).
 //
-// tcgen05 MMAs issued by one thread execute in issue order, and a commit
-// arrives once every earlier MMA of the thread has completed; so S_{h+2} may
-// overwrite the P_h that PV_h reads (it is issued after it).  The softmax
-// rescales O only after the P V of the previous half-tile has completed.
+// Ordering of the MMAs.  S_{h+2} overwrites the TMEM buffer whose P the P V of
+// half-tile h reads.  The PTX ISA orders two asynchronous tcgen05 operations of
+// one thread only for the pairs it lists as tcgen05 pipelines ("pipelined
+// tcgen05 instructions"): MMA -> MMA only for the same accumulator and shape,
+// but MMA -> shift and shift -> MMA for any two of the same cta_group.  So
+// before S_{h+2} the MMA lane issues a tcgen05.shift of one 32-byte column
+// group of that buffer: P V_h -> shift -> S_{h+2} is a chain of listed pairs,
+// the shift only disturbs columns that S_{h+2} then overwrites (its first MMA
+// does not accumulate), and no thread waits.  The softmax rescales O only after
+// the P V of the previous half-tile has completed.
+//
+// Work order.  CTA x takes query tile qorder[x] of its head (the mask's
+// dispatch order; identity when absent): query tiles sorted by in-frame
+// position band, then frame, so that the CTAs resident together share a
+// position band across many frames and walk overlapping key tiles of every
+// frame (eq. 4's bands are centred on the query's own in-frame position).
 //
 // Online softmax in base 2: x = S * scale * log2(e); p = 2^(x - m) with m a
 // running maximum that is only raised (and O, l rescaled) when a half-tile's
@@ -67,7 +79,9 @@ constexpr float RESCALE_THRESHOLD = 8.0f;
 // Wait-site codes recorded with a timeout.
 enum : int {
     SITE_Q_FULL = 1, SITE_K_EMPTY, SITE_V_EMPTY, SITE_K_FULL, SITE_P_FULL, SITE_V_FULL, SITE_S_FULL,
-    SITE_PV_DONE, SITE_O_FINAL, SITE_SELFTEST, SITE_SMEM_ALIGN
+    SITE_PV_DONE, SITE_O_FINAL, SITE_SELFTEST, SITE_SMEM_ALIGN,
+    // bounds checks of the debug build
+    SITE_B_QTILE = 40, SITE_B_ROW, SITE_B_KTILE, SITE_B_SELFTEST
 };
 
 template <int D>
@@ -110,35 +124,14 @@ struct FwdParams {
     const int* row_ptr;
     const int* col_idx;
     const unsigned char* flag;
+    const int* qorder; // query tile of CTA x (a permutation of [0, nb)), or null for x itself
+    int nnz;           // entries of col_idx / flag (bounds checks of the debug build)
     __nv_bfloat16* O;
     float* lse;
     float scale_log2;  // scale * log2(e)
     unsigned long long timeout_ns;
 };
 
-// ---- packed fp32 pairs (sm_100 f32x2 instructions) -------------------------
-__device__ __forceinline__ uint64_t f2pack(float lo, float hi)
-{
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi)
-{
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c)
-{
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b)
-{
-    uint64_t d;
-    asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
 __device__ __forceinline__ float max3(float a, float b, float c)
 {
     float d;
@@ -146,70 +139,23 @@ __device__ __forceinline__ float max3(float a, float b, float c)
     return d;
 }
 
-// 2^x for a pair of values on the FMA pipe instead of MUFU.  Range reduction
-// x = j + f with j = round(x) (by the 1.5 * 2^23 rounding constant) and
-// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial (Remez fit of the relative
-// error, coefficients from exp2_poly_fit.py, max relative error 7.5e-5); 2^j
-// added to the exponent field.  x is clamped at -126, so the result is
-// a tiny positive number (not 0) below 2^-126: only used on unmasked tiles.
-constexpr float EXP2_C0 = 0.99992806f, EXP2_C1 = 0.69326097f, EXP2_C2 = 0.24261113f, EXP2_C3 = 0.05517167f;
-__device__ __forceinline__ void poly_exp2_x2(float x0, float x1, float& y0, float& y1)
-{
-    const float rnd = 12582912.0f;  // 1.5 * 2^23
-    x0 = fmaxf(x0, -126.0f);
-    x1 = fmaxf(x1, -126.0f);
-    const uint64_t x = f2pack(x0, x1);
-    const uint64_t r = f2add(x, f2pack(rnd, rnd));               // j in the low mantissa bits
-    const uint64_t j = f2add(r, f2pack(-rnd, -rnd));
-    const uint64_t f = f2fma(j, f2pack(-1.0f, -1.0f), x);         // x - j
-    uint64_t poly = f2fma(f2pack(EXP2_C3, EXP2_C3), f, f2pack(EXP2_C2, EXP2_C2));
-    poly = f2fma(poly, f, f2pack(EXP2_C1, EXP2_C1));
-    poly = f2fma(poly, f, f2pack(EXP2_C0, EXP2_C0));
-    float p0, p1, r0, r1;
-    f2unpack(poly, p0, p1);
-    f2unpack(r, r0, r1);
-    // (bits of r) << 23 == j << 23 modulo 2^32, since 0x4B400000 << 23 wraps to 0.
-    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(r0) << 23));
-    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(r1) << 23));
-}
-
 // Exponentials, bf16 packing and row sums of one 32-column chunk of S:
-// p = 2^(s * c - m).  The first EMU elements of the chunk use the polynomial,
-// the rest MUFU ex2.  The row sum is kept in SUMACC independent accumulators
-// (short dependency chains).  SPLIT also returns the bf16 residuals.
-#ifndef RA_SUMACC
-#define RA_SUMACC 8
-#endif
-#ifndef RA_MAXACC
-#define RA_MAXACC 8
-#endif
-#ifndef RA_FFMA2
-#define RA_FFMA2 0
-#endif
-template <int EMU, bool SPLIT, bool MAX>
-__device__ __forceinline__ void exp_chunk(const uint32_t (&r)[32], float c, float negm, float (&acc)[RA_SUMACC],
+// p = 2^(s * c - m) on MUFU ex2.  The row sum is kept in SUM_ACC independent
+// accumulators (short dependency chains).  SPLIT also returns the bf16
+// residuals; MAX also tracks the raw maximum of the chunk.
+constexpr int SUM_ACC = 8;
+constexpr int MAX_ACC = 8;
+template <bool SPLIT, bool MAX>
+__device__ __forceinline__ void exp_chunk(const uint32_t (&r)[32], float c, float negm, float (&acc)[SUM_ACC],
                                           float (&mx)[4], uint32_t (&pk)[16], uint32_t (&pl)[16])
 {
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
         if (MAX)
             mx[(e >> 1) & 3] = max3(mx[(e >> 1) & 3], __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
-        float x0, x1, p0, p1;
-        if (RA_FFMA2) {
-            const uint64_t x2 = f2fma(f2pack(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), f2pack(c, c),
-                                      f2pack(negm, negm));
-            f2unpack(x2, x0, x1);
-        } else {
-            x0 = fmaf(__uint_as_float(r[e]), c, negm);
-            x1 = fmaf(__uint_as_float(r[e + 1]), c, negm);
-        }
-        if (e < EMU) {
-            poly_exp2_x2(x0, x1, p0, p1);
-        } else {
-            p0 = fast_exp2(x0);
-            p1 = fast_exp2(x1);
-        }
-        acc[(e >> 1) % RA_SUMACC] += p0 + p1;
+        const float p0 = fast_exp2(fmaf(__uint_as_float(r[e]), c, negm));
+        const float p1 = fast_exp2(fmaf(__uint_as_float(r[e + 1]), c, negm));
+        acc[(e >> 1) % SUM_ACC] += p0 + p1;
         pk[e >> 1] = pack_bf16(p0, p1);
         if (SPLIT) {
             const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&pk[e >> 1]);
@@ -217,14 +163,6 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&r)[32], float c, floa
         }
     }
 }
-
-// Elements of each 32-column chunk whose exponential runs on the FMA pipe
-// (unmasked tiles, bf16 P only): shifts work off the MUFU unit, which at
-// d = 128 needs as many cycles per tile as the tensor core.
-#ifndef RA_EMU_PER_32
-#define RA_EMU_PER_32 0
-#endif
-constexpr int EMU_PER_32 = RA_EMU_PER_32;
 
 // SPLIT_P: P is kept as hi + lo bf16 pairs (P = hi + lo to ~16 bits) and
 // P V runs as two MMAs; used for masks whose rows hold few keys, where the
@@ -244,7 +182,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::BAR_OFF + 8 * B_COUNT + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int qb = p.qorder ? p.qorder[blockIdx.x] : static_cast<int>(blockIdx.x);
+    const int h = blockIdx.y, b = blockIdx.z;
     const int bh = b * p.H + h;
     const int n = p.g.n;
     WaitCtl wc{abort_flag, g_err, p.timeout_ns};
@@ -253,6 +192,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
         *abort_flag = *reinterpret_cast<volatile int*>(g_err) != 0 ? 1 : 0;
         if (sbase & 1023u)  // the swizzled tiles need 1024-byte alignment: record it, run nothing
             report_timeout(wc, SITE_SMEM_ALIGN);
+        // (debug build) the query tile and its CSR row are in range
+        if (!*abort_flag && in_bounds(wc, qb >= 0 && qb < p.nb, SITE_B_QTILE))
+            in_bounds(wc, 0 <= p.row_ptr[qb] && p.row_ptr[qb] <= p.row_ptr[qb + 1] && p.row_ptr[qb + 1] <= p.nnz,
+                      SITE_B_ROW);
         for (int i = 0; i < B_COUNT; ++i)
             mbar_init(bar(i), (i == B_P_FULL || i == B_P_FULL + 1) ? 128u : 1u);
         fence_barrier_init();
@@ -268,7 +211,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     const uint32_t tmem = *tmem_slot;
     const bool skip = *abort_flag != 0;  // an earlier CTA gave up: do nothing
 
-    const int row_start = p.row_ptr[qb];
+    const int row_start = skip ? 0 : p.row_ptr[qb];
     const int L_row = skip ? 0 : p.row_ptr[qb + 1] - row_start;
     const int n_half = 2 * L_row;
 
@@ -283,7 +226,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
                 tma_load_3d(sQ + c * L::Q_CHUNK_BYTES, &tmQ, bar(B_Q_FULL), c * 64, qb * TILE, bh);
             int k_issued = 0, v_issued = 0;
             for (int hh = 0; hh < n_half; ++hh) {
-                const int key0 = p.col_idx[row_start + (hh >> 1)] * TILE + (hh & 1) * HALF;
+                const int kb = p.col_idx[row_start + (hh >> 1)];
+                if (!in_bounds(wc, kb >= 0 && kb < p.nbk, SITE_B_KTILE))  // (debug build)
+                    break;
+                const int key0 = kb * TILE + (hh & 1) * HALF;
                 const int ks = hh % L::KS, vs = hh % L::VS;
                 if (hh >= L::KS && !mbar_wait(bar(B_K_EMPTY + ks), ((hh / L::KS) - 1) & 1, wc, SITE_K_EMPTY))
                     break;
@@ -336,6 +282,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
                     if (!(ok = wait_all(bar(B_K_FULL + ks), (hh / L::KS) & 1, SITE_K_FULL)))
                         break;
                     tc_fence_after();
+                    // Order S_hh after that P V: MMA -> shift -> MMA (see the header).
+                    if (hh >= 2 && leader)
+                        tmem_shift_down(tmem + s_col_of(hh & 1));
                     const uint64_t kd = desc_add(k_desc, ks * L::H_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
@@ -446,31 +395,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
             // Exponentials of the half-tile against m_use, P to TMEM; with
             // fused_max the same pass also finds the half-tile's raw maximum.
             auto exp_pass = [&](float m_use, bool fused_max, float& mx_out) -> float {
-                float acc[RA_SUMACC];
+                float acc[SUM_ACC];
 #pragma unroll
-                for (int a = 0; a < RA_SUMACC; ++a)
+                for (int a = 0; a < SUM_ACC; ++a)
                     acc[a] = 0.f;
                 float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     uint32_t pk[16], pl[16];
-                    if (SPLIT_P || masked) {
-                        if (fused_max)
-                            exp_chunk<0, SPLIT_P, true>(r[c], p.scale_log2, -m_use, acc, mx, pk, pl);
-                        else
-                            exp_chunk<0, SPLIT_P, false>(r[c], p.scale_log2, -m_use, acc, mx, pk, pl);
-                    } else {
-                        if (fused_max)
-                            exp_chunk<EMU_PER_32, false, true>(r[c], p.scale_log2, -m_use, acc, mx, pk, pl);
-                        else
-                            exp_chunk<EMU_PER_32, false, false>(r[c], p.scale_log2, -m_use, acc, mx, pk, pl);
-                    }
+                    if (fused_max)
+                        exp_chunk<SPLIT_P, true>(r[c], p.scale_log2, -m_use, acc, mx, pk, pl);
+                    else
+                        exp_chunk<SPLIT_P, false>(r[c], p.scale_log2, -m_use, acc, mx, pk, pl);
                     tmem_st16(lane_base + s_col + c * 16, pk);
                     if (SPLIT_P)
                         tmem_st16(lane_base + s_col + HALF / 2 + c * 16, pl);
                 }
 #pragma unroll
-                for (int w = RA_SUMACC / 2; w >= 1; w /= 2)
+                for (int w = SUM_ACC / 2; w >= 1; w /= 2)
 #pragma unroll
                     for (int a = 0; a < w; ++a)
                         acc[a] += acc[a + w];
@@ -507,15 +449,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
             float sum, mx_raw;
             if (__any_sync(0xFFFFFFFFu, m_run == -INFINITY)) {
                 // No reference maximum yet in this warp: the max first, then the pass.
-                float mc[RA_MAXACC];
+                float mc[MAX_ACC];
 #pragma unroll
-                for (int a = 0; a < RA_MAXACC; ++a)
+                for (int a = 0; a < MAX_ACC; ++a)
                     mc[a] = -INFINITY;
 #pragma unroll
                 for (int idx = 0; idx < HALF; ++idx)
-                    mc[idx % RA_MAXACC] = fmaxf(mc[idx % RA_MAXACC], __uint_as_float(r[idx / 32][idx % 32]));
+                    mc[idx % MAX_ACC] = fmaxf(mc[idx % MAX_ACC], __uint_as_float(r[idx / 32][idx % 32]));
 #pragma unroll
-                for (int w = RA_MAXACC / 2; w >= 1; w /= 2)
+                for (int w = MAX_ACC / 2; w >= 1; w /= 2)
 #pragma unroll
                     for (int a = 0; a < w; ++a)
                         mc[a] = fmaxf(mc[a], mc[a + w]);
@@ -601,6 +543,19 @@ __global__ void wait_selftest_kernel(unsigned long long timeout_ns)
     }
 }
 
+#ifdef RA_DEBUG_BOUNDS
+// Bounds-check self-test: one thread fails a check on an index it never uses.
+__global__ void bounds_selftest_kernel()
+{
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        WaitCtl wc{&abort_flag, g_err, 0};
+        in_bounds(wc, false, SITE_B_SELFTEST);
+    }
+}
+#endif
+
 template <int D, bool SPLIT_P>
 ra_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p, int B,
                      cudaStream_t cs)
@@ -684,6 +639,8 @@ extern "C" ra_status ra_attention_fwd(const void* Q, const void* K, const void* 
     p.row_ptr = m->row_ptr;
     p.col_idx = m->col_idx;
     p.flag = m->flag;
+    p.qorder = m->qorder;
+    p.nnz = static_cast<int>(m->nnz);
     p.O = static_cast<__nv_bfloat16*>(O);
     p.lse = lse;
     p.scale_log2 = scale * 1.4426950408889634f;
@@ -701,7 +658,7 @@ extern "C" ra_status ra_attention_fwd(const void* Q, const void* K, const void* 
 namespace ra {
 ra_status attention_fwd_rect(const void* Q, const void* K, const void* V, void* O, int B, int H, int d, int nq,
                              int nk, int k_head_rows, const int* row_ptr, const int* col_idx,
-                             const unsigned char* flag, int nbq, float scale, float* lse, cudaStream_t cs)
+                             const unsigned char* flag, int nbq, int nnz, float scale, float* lse, cudaStream_t cs)
 {
     ra_status st;
     CUtensorMap mq, mk, mv;
@@ -724,6 +681,7 @@ ra_status attention_fwd_rect(const void* Q, const void* K, const void* V, void* 
     p.row_ptr = row_ptr;
     p.col_idx = col_idx;
     p.flag = flag;
+    p.nnz = nnz;
     p.O = static_cast<__nv_bfloat16*>(O);
     p.lse = lse;
     p.scale_log2 = scale * 1.4426950408889634f;
@@ -802,6 +760,22 @@ extern "C" ra_status ra_selftest_wait_timeout(long long timeout_ns, ra_stream st
     wait_selftest_kernel<<<1, 32, 0, cs>>>(static_cast<unsigned long long>(timeout_ns));
     RA_CUDA_TRY(cudaGetLastError());
     return ra_get_device_status(stream);
+}
+
+extern "C" ra_status ra_selftest_bounds(ra_stream stream)
+{
+#ifdef RA_DEBUG_BOUNDS
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    ra_status st = ra_get_device_status(stream);  // start from a clean word
+    if (st != RA_OK && st != RA_ERR_DEVICE_TIMEOUT && st != RA_ERR_DEVICE_BOUNDS)
+        return st;
+    bounds_selftest_kernel<<<1, 32, 0, cs>>>();
+    RA_CUDA_TRY(cudaGetLastError());
+    return ra_get_device_status(stream);
+#else
+    (void)stream;
+    return fail(RA_ERR_UNSUPPORTED, "bounds checks are compiled only into the debug library (-DRA_DEBUG_BOUNDS)");
+#endif
 }
 
 extern "C" ra_status ra_set_pv_precision(int policy)

@@ -37,7 +37,9 @@ constexpr uint32_t BWD_TMEM_COLS = 512;
 constexpr float LOG2E = 1.4426950408889634f;
 
 enum : int { BSITE_RES = 21, BSITE_X_EMPTY, BSITE_Y_EMPTY, BSITE_X_FULL, BSITE_Y_FULL, BSITE_S_FULL, BSITE_DS_FULL,
-             BSITE_ACC, BSITE_FINAL };
+             BSITE_ACC, BSITE_FINAL,
+             // bounds checks of the debug build
+             BSITE_B_ROW = 50, BSITE_B_TILE };
 
 struct BwdParams {
     MaskGeom g;
@@ -45,6 +47,7 @@ struct BwdParams {
     const int* ptr;            // row_ptr (dQ pass) or col_ptr (dK/dV pass)
     const int* idx;            // col_idx or row_idx
     const unsigned char* flag; // flag or tflag
+    int nnz;                   // entries of idx / flag (bounds checks of the debug build)
     const float* lse;          // [B*H, n] natural log
     const float* Dv;           // [B*H, n] rowsum(dO * O)
     __nv_bfloat16* out0;       // dQ, or dK
@@ -154,8 +157,10 @@ __device__ __forceinline__ void mask_chunk(uint32_t (&s)[32], uint32_t keep)
 // dP = dO V^T are computed for a whole 128-key tile per step.  TMEM: S in two
 // buffers (columns 0 and 128), dP in one (256; the gradient warps load it into
 // registers first and release it at once), dQ at 384.  The MMA warp issues
-// dP_j, then S_j, then the gradient MMA of step j - 1, so that its wait for the
-// gradient MMA of step j - 2 (whose dS buffer S_j overwrites) overlaps dP_j.
+// dP_j, then S_j, then the gradient MMA of step j - 1.  S_j overwrites the dS
+// that the gradient MMA of step j - 2 reads; a tcgen05.shift on that buffer
+// between the two orders them (MMA -> shift -> MMA are pipelined pairs of the
+// PTX ISA, executed in issue order), with no wait.
 // 320 threads: two gradient warpgroups (columns 64 wg .. 64 wg + 63 of each
 // step), warp 8 issues the TMA loads, warp 9 the MMAs.
 constexpr int DQ_THREADS = 320, DQ_GRAD_THREADS = 256, DQ_PRODUCER_WARP = 8, DQ_MMA_WARP = 9;
@@ -187,8 +192,7 @@ struct DqBars {
     static constexpr int S_FULL = V_EMPTY + VS;  // + buffer: S_j and dP_j complete
     static constexpr int DP_FREE = S_FULL + 2;   // the gradient warps have loaded dP
     static constexpr int DS_FULL = DP_FREE + 1;  // + buffer: dS of the step written
-    static constexpr int ACC_DONE = DS_FULL + 2; // + buffer: dQ += dS K of the step complete
-    static constexpr int FINAL = ACC_DONE + 2;
+    static constexpr int FINAL = DS_FULL + 2;
     static constexpr int COUNT = FINAL + 1;
 };
 
@@ -224,6 +228,9 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
         }
         fence_barrier_init();
         fence_proxy_async_smem();
+        // (debug build) this tile's CSR row is in range
+        if (!*abort_flag)
+            in_bounds(wc, 0 <= p.ptr[qb] && p.ptr[qb] <= p.ptr[qb + 1] && p.ptr[qb + 1] <= p.nnz, BSITE_B_ROW);
     }
     if (warp == DQ_MMA_WARP) {
         tmem_alloc(smem_addr(tmem_slot), BWD_TMEM_COLS);
@@ -234,7 +241,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const bool skip = *abort_flag != 0;
-    const int start = p.ptr[qb];
+    const int start = skip ? 0 : p.ptr[qb];
     const int len = skip ? 0 : p.ptr[qb + 1] - start;
 
     if (warp == DQ_PRODUCER_WARP) {
@@ -247,7 +254,10 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
             }
             int k_issued = 0, v_issued = 0;
             for (int j = 0; j < len; ++j) {
-                const int row0 = p.idx[start + j] * TILE;
+                const int tile = p.idx[start + j];
+                if (!in_bounds(wc, tile >= 0 && tile < p.nb, BSITE_B_TILE))  // (debug build)
+                    break;
+                const int row0 = tile * TILE;
                 const int ks = j % L::KS, vs = j % L::VS;
                 if (j >= L::VS && !mbar_wait(bar(BB::V_EMPTY + vs), ((j / L::VS) - 1) & 1, wc, BSITE_Y_EMPTY))
                     break;
@@ -296,7 +306,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
             // dQ += dS_j K_j: dS packed by the warpgroups, keys 16 kk .. 16 kk + 15
             // at columns 64 (kk / 4) + 8 (kk % 4) of the step's S buffer.
             auto issue_acc = [&](int j) {
-                const int bf = j & 1, ks = j % L::KS;
+                const int bf = j & 1, ks = j % L::KS;  // dS_j in S buffer bf
                 const uint64_t kdesc = desc_add(dKmn, ks * L::TILE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < TILE / 16; ++kk) {
@@ -305,10 +315,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
                         mma_ts(tmem + DQ_COL_ACC, tmem + dq_s_col(bf) + (kk >> 2) * 64 + (kk & 3) * 8, bd, idesc_acc,
                                (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                if (leader) {
-                    mma_commit(bar(BB::ACC_DONE + bf));
+                if (leader)
                     mma_commit(bar(BB::K_EMPTY + ks));
-                }
             };
             auto wait_all = [&](uint32_t b, uint32_t parity, int site) {
                 return __all_sync(0xFFFFFFFFu, mbar_wait(b, parity, wc, site));
@@ -327,14 +335,14 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
                 mma_s(DQ_COL_DP, dOd, desc_add(dVd, vs * L::TILE_BYTES));
                 if (leader)
                     mma_commit(bar(BB::V_EMPTY + vs));
-                // S_j into buffer bf, once the gradient MMA of step j - 2 (which read
-                // dS from that buffer) has completed: MMAs into different
-                // accumulators are not ordered
+                // S_j into buffer bf, after the gradient MMA of step j - 2 that
+                // reads dS from it: MMAs into different accumulators are not
+                // ordered, MMA -> shift -> MMA is
                 if (!(ok = wait_all(bar(BB::K_FULL + ks), (j / L::KS) & 1, BSITE_X_FULL)))
                     break;
-                if (j >= 2 && !(ok = wait_all(bar(BB::ACC_DONE + bf), ((j - 2) >> 1) & 1, BSITE_ACC)))
-                    break;
                 tc_fence_after();
+                if (j >= 2 && leader)
+                    tmem_shift_down(tmem + dq_s_col(bf));
                 mma_s(dq_s_col(bf), dQd, desc_add(dKd, ks * L::TILE_BYTES));
                 if (leader)
                     mma_commit(bar(BB::S_FULL + bf));
@@ -482,11 +490,15 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
 // dP^T (128; dS^T is packed back over its first half), dK (256) and dV (384),
 // so P^T, the A operand of dV += P^T dO, goes to shared memory in the
 // 128-byte-swizzled K-major layout.  Per step j the MMA warp issues S^T_{j+1}
-// as soon as the gradient warps have loaded S^T_j and dP^T_j into registers,
-// then dK_j and dV_j, then dP^T_{j+1} once dK_j (which reads dS^T from the
-// dP^T columns) has completed; dV_j runs meanwhile.  320 threads: two
-// gradient warpgroups (query columns 64 wg .. 64 wg + 63 of each step), warp
-// 8 issues the TMA loads, warp 9 the MMAs.
+// as soon as the gradient warps have loaded S^T_j and dP^T_j into registers;
+// the half of dK_j that reads the first 32-column chunk of each warpgroup's
+// dS^T as soon as those chunks are written (while the gradient warps work on
+// their second chunks), the other half when the step's dS^T is complete; then
+// dP^T_{j+1} over the dS^T columns, ordered after dK_j by a tcgen05.shift
+// (MMA -> shift -> MMA are pipelined pairs of the PTX ISA, executed in issue
+// order), with no wait; then dV_j.  320 threads: two gradient warpgroups
+// (query columns 64 wg .. 64 wg + 63 of each step), warp 8 issues the TMA
+// loads, warp 9 the MMAs.
 constexpr int KV_THREADS = 320, KV_GRAD_THREADS = 256, KV_PRODUCER_WARP = 8, KV_MMA_WARP = 9;
 constexpr uint32_t KV_COL_S = 0, KV_COL_DP = 128, KV_COL_DK = 256, KV_COL_DV = 384;
 
@@ -519,8 +531,8 @@ struct KvBars {
     static constexpr int S_FULL = O_EMPTY + OS;  // S^T_j and dP^T_j complete (and every earlier MMA)
     static constexpr int S_FREE = S_FULL + 1;    // the gradient warps have loaded S^T_j and dP^T_j
     static constexpr int DS_FULL = S_FREE + 1;   // P^T_j (shared memory) and dS^T_j (TMEM) written
-    static constexpr int DK_DONE = DS_FULL + 1;  // dK += dS^T_j Q_j complete
-    static constexpr int DV_DONE = DK_DONE + 1;  // dV += P^T_j dO_j complete (P^T may be overwritten)
+    static constexpr int DS_HALF = DS_FULL + 1;  // the first 32-column chunk of each warpgroup's dS^T_j written
+    static constexpr int DV_DONE = DS_HALF + 1;  // dV += P^T_j dO_j complete (P^T may be overwritten)
     static constexpr int FINAL = DV_DONE + 1;
     static constexpr int COUNT = FINAL + 1;
 };
@@ -556,11 +568,14 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
     if (threadIdx.x == 0) {
         *abort_flag = *reinterpret_cast<volatile int*>(p.err) != 0 ? 1 : 0;
         for (int i = 0; i < BB::COUNT; ++i) {
-            const bool grad = i == BB::S_FREE || i == BB::DS_FULL;
+            const bool grad = i == BB::S_FREE || i == BB::DS_FULL || i == BB::DS_HALF;
             mbar_init(bar(i), grad ? static_cast<uint32_t>(KV_GRAD_THREADS) : 1u);
         }
         fence_barrier_init();
         fence_proxy_async_smem();
+        // (debug build) this tile's CSR row is in range
+        if (!*abort_flag)
+            in_bounds(wc, 0 <= p.ptr[kb] && p.ptr[kb] <= p.ptr[kb + 1] && p.ptr[kb + 1] <= p.nnz, BSITE_B_ROW);
     }
     if (warp == KV_MMA_WARP) {
         tmem_alloc(smem_addr(tmem_slot), BWD_TMEM_COLS);
@@ -571,7 +586,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const bool skip = *abort_flag != 0;
-    const int start = p.ptr[kb];
+    const int start = skip ? 0 : p.ptr[kb];
     const int len = skip ? 0 : p.ptr[kb + 1] - start;
 
     if (warp == KV_PRODUCER_WARP) {
@@ -584,7 +599,10 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
             }
             int q_issued = 0, o_issued = 0;
             for (int j = 0; j < len; ++j) {
-                const int row0 = p.idx[start + j] * TILE;
+                const int tile = p.idx[start + j];
+                if (!in_bounds(wc, tile >= 0 && tile < p.nb, BSITE_B_TILE))  // (debug build)
+                    break;
+                const int row0 = tile * TILE;
                 const int qs = j % L::QS, os = j % L::OS;
                 if (j >= L::QS && !mbar_wait(bar(BB::Q_EMPTY + qs), ((j / L::QS) - 1) & 1, wc, BSITE_X_EMPTY))
                     break;
@@ -633,21 +651,22 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                 }
             };
             // dK += dS^T_j Q_j: dS^T packed by the warpgroups, queries 16 kk .. 16 kk + 15
-            // at columns 64 (kk / 4) + 8 (kk % 4) of the dP^T buffer.
-            auto issue_dk = [&](int j) {
+            // at columns 64 (kk / 4) + 8 (kk % 4) of the dP^T buffer.  Half h of
+            // the products: kk = 4 wg + 2 h + {0, 1}, the h-th 32-column chunk of
+            // each warpgroup; the Q tile is released after the second half.
+            auto issue_dk = [&](int j, int half) {
                 const int qs = j % L::QS;
                 const uint64_t qdesc = desc_add(dQmn, qs * L::TILE_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < TILE / 16; ++kk) {
+                for (int u = 0; u < 4; ++u) {
+                    const int kk = 4 * (u >> 1) + 2 * half + (u & 1);
                     const uint64_t bd = desc_add(qdesc, kk * 2048);
                     if (leader)
                         mma_ts(tmem + KV_COL_DK, tmem + KV_COL_DP + (kk >> 2) * 64 + (kk & 3) * 8, bd, idesc_acc,
                                (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                if (leader) {
-                    mma_commit(bar(BB::DK_DONE));
+                if (leader && half == 1)
                     mma_commit(bar(BB::Q_EMPTY + qs));
-                }
             };
             // dV += P^T_j dO_j: P^T from shared memory (K-major over the queries).
             auto issue_dv = [&](int j) {
@@ -690,19 +709,24 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                     tc_fence_after();
                     mma_s(KV_COL_S, dKd, desc_add(dQd, (jn % L::QS) * L::TILE_BYTES));
                 }
+                if (!(ok = wait_all(bar(BB::DS_HALF), j & 1, BSITE_DS_FULL)))
+                    break;
+                tc_fence_after();
+                issue_dk(j, 0);
                 if (!(ok = wait_all(bar(BB::DS_FULL), j & 1, BSITE_DS_FULL)))
                     break;
                 tc_fence_after();
-                issue_dk(j);
+                issue_dk(j, 1);
                 if (jn < len) {
-                    // dP^T_{j+1} over the dS^T_j that dK_j read: once dK_j has
-                    // completed (MMAs into different accumulators are not
-                    // ordered), and ahead of dV_j, so that the next step's
-                    // gradient warps start sooner
-                    if (!(ok = wait_all(bar(BB::O_FULL + jn % L::OS), (jn / L::OS) & 1, BSITE_Y_FULL)) ||
-                        !(ok = wait_all(bar(BB::DK_DONE), j & 1, BSITE_ACC)))
+                    // dP^T_{j+1} over the dS^T_j that dK_j reads, ordered after
+                    // dK_j by MMA -> shift -> MMA (MMAs into different
+                    // accumulators are not ordered), and ahead of dV_j, so that
+                    // the next step's gradient warps start sooner
+                    if (!(ok = wait_all(bar(BB::O_FULL + jn % L::OS), (jn / L::OS) & 1, BSITE_Y_FULL)))
                         break;
                     tc_fence_after();
+                    if (leader)
+                        tmem_shift_down(tmem + KV_COL_DP);
                     mma_s(KV_COL_DP, dVd, desc_add(dOd, (jn % L::OS) * L::TILE_BYTES));
                     if (leader)
                         mma_commit(bar(BB::S_FULL));
@@ -731,6 +755,8 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
         // there), threads 64-127 -D.  Loaded one step ahead of its use, with the
         // CSR entry.
         auto column_stat = [&](int qblock) -> float {
+            if (!in_bounds(wc, qblock >= 0 && qblock < p.nb, BSITE_B_TILE))  // (debug build)
+                return -INFINITY;
             const int q = qblock * TILE + static_cast<int>(my_col) + (t & 63);
             if (q >= n)
                 return t < 64 ? -INFINITY : -0.f;
@@ -815,6 +841,12 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                 }
                 // dS^T packed over dP^T columns this warpgroup has already loaded
                 tmem_st16(lane_base + KV_COL_DP + my_col + c * 16, dk);
+                if (c == 0) {
+                    // the first chunk's dS^T: its half of dK_j can start
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar(BB::DS_HALF));
+                }
             }
             tmem_wait_st();
             fence_proxy_async_smem();  // P^T is read by the tensor cores
@@ -947,6 +979,7 @@ ra_status run_bwd(const void* Q, const void* K, const void* V, const void* O, co
     p.nb = m->nb;
     p.H = H;
     p.mode = mode;
+    p.nnz = static_cast<int>(m->nnz);
     p.lse = lse;
     p.Dv = Dws;
     p.scale = scale;
@@ -989,6 +1022,13 @@ extern "C" ra_status ra_attention_bwd(const void* Q, const void* K, const void* 
     }
     if (!lse || !D_workspace)
         return fail(RA_ERR_INVALID_ARG, "NULL lse or workspace");
+    {
+        const void* all[10] = {Q, K, V, O, dO, lse, dQ, dK, dV, D_workspace};
+        for (int i = 6; i < 10; ++i)
+            for (int j = 0; j < 10; ++j)
+                if (j != i && all[i] == all[j])
+                    return fail(RA_ERR_INVALID_ARG, "outputs (dQ, dK, dV, D_workspace) may not alias another buffer");
+    }
     if (!m)
         return fail(RA_ERR_INVALID_ARG, "NULL mask");
     if (B < 1 || H < 1 || B > 65535 || H > 65535)
@@ -1001,6 +1041,21 @@ extern "C" ra_status ra_attention_bwd(const void* Q, const void* K, const void* 
         return fail(RA_ERR_INVALID_ARG, "scale must be finite and > 0");
     if (m->nnz == 0 || !m->col_ptr)
         return fail(RA_ERR_INVALID_ARG, "mask has no kept tile");
+    // dQ is written before the dK / dV kernel reads Q and dO, and D before it is
+    // read with lse: an output overlapping any other buffer would corrupt the
+    // result silently, so every output range must be disjoint from the rest.
+    const size_t tbytes = static_cast<size_t>(B) * H * m->geom.n * d * 2;
+    const size_t sbytes = static_cast<size_t>(B) * H * m->geom.n * sizeof(float);
+    const void* bufs[10] = {Q, K, V, O, dO, lse, dQ, dK, dV, D_workspace};
+    const size_t sizes[10] = {tbytes, tbytes, tbytes, tbytes, tbytes, sbytes, tbytes, tbytes, tbytes, sbytes};
+    auto overlap = [&](int i, int j) {
+        const uintptr_t a = reinterpret_cast<uintptr_t>(bufs[i]), b = reinterpret_cast<uintptr_t>(bufs[j]);
+        return a < b + sizes[j] && b < a + sizes[i];
+    };
+    for (int i = 6; i < 10; ++i)
+        for (int j = 0; j < 10; ++j)
+            if (j != i && overlap(i, j))
+                return fail(RA_ERR_INVALID_ARG, "outputs (dQ, dK, dV, D_workspace) may not overlap any other buffer");
     int dev = 0;
     RA_CUDA_TRY(cudaGetDevice(&dev));
     if (dev != m->device)

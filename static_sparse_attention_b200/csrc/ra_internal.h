@@ -24,6 +24,9 @@ struct ra_mask {
     int* col_ptr;
     int* row_idx;
     unsigned char* tflag;
+    // Dispatch order of the forward's query tiles (CTA x runs query tile
+    // qorder[x]); null when it is the identity.
+    int* qorder;
 };
 
 namespace ra {
@@ -52,7 +55,8 @@ ra_status make_map_rows(CUtensorMap* map, const void* base, int BH, int rows, in
 // every listed key, such as the window held by the SWC key/value cache.
 ra_status attention_fwd_rect(const void* Q, const void* K, const void* V, void* O, int B, int H, int d, int nq,
                              int nk, int k_head_rows, const int* row_ptr, const int* col_idx,
-                             const unsigned char* flag, int nbq, float scale, float* lse, cudaStream_t stream);
+                             const unsigned char* flag, int nbq, int nnz, float scale, float* lse,
+                             cudaStream_t stream);
 
 // Device address of the forward / backward kernels' error word on the current device.
 ra_status device_error_word(int** out);

@@ -19,7 +19,9 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
-#include <mutex>
+#include <algorithm>
+#include <utility>
+#include <vector>
 
 #include "ra_internal.h"
 
@@ -247,6 +249,34 @@ __global__ void __launch_bounds__(128) col_compact_kernel(const int* __restrict_
     }
 }
 
+// The order in which the forward's CTAs take query tiles: sorted by in-frame
+// position band, then by frame.  eq. 4 keeps, in every key frame, a band of
+// positions centred on the query's own in-frame position, so query tiles of one
+// position band over many frames read overlapping key tiles; with the query
+// tiles of a head in plain order the resident CTAs instead cover a few whole
+// frames, i.e. every position, and at long sequences (a head's K and V well
+// beyond the L2 cache) re-read most key tiles from DRAM.  A band holds about
+// three query tiles per SM (1.5 times the forward's resident CTAs); masks of a
+// few such bands, and frames shorter than two tiles, keep the plain order.
+// Returns false when the order is the identity.
+bool dispatch_order(const MaskGeom& g, int nb, int sm_count, std::vector<int>& order)
+{
+    const long long per_band = 3LL * (sm_count > 0 ? sm_count : 148);
+    const int bands = static_cast<int>((nb + per_band / 2) / per_band);
+    if (g.s < 2 * TILE || bands < 2)
+        return false;
+    order.resize(nb);
+    for (int q = 0; q < nb; ++q)
+        order[q] = q;
+    auto key = [&](int q) {
+        const long long first = static_cast<long long>(q) * TILE;
+        const long long band = (first % g.s) * bands / g.s;
+        return std::make_pair(band, first / g.s);
+    };
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return key(a) < key(b); });
+    return true;
+}
+
 void free_mask_arrays(ra_mask* m)
 {
     cudaFree(m->row_ptr);
@@ -256,7 +286,8 @@ void free_mask_arrays(ra_mask* m)
     cudaFree(m->col_ptr);
     cudaFree(m->row_idx);
     cudaFree(m->tflag);
-    m->row_ptr = m->col_idx = m->count = m->col_ptr = m->row_idx = nullptr;
+    cudaFree(m->qorder);
+    m->row_ptr = m->col_idx = m->count = m->col_ptr = m->row_idx = m->qorder = nullptr;
     m->flag = m->tflag = nullptr;
 }
 
@@ -404,6 +435,17 @@ extern "C" ra_status ra_build_mask(int family, int f, int s, const ra_mask_param
         if ((e = cudaGetLastError()) != cudaSuccess)
             return bail(e, "col_compact_kernel launch");
     }
+    int sm_count = 0;
+    if ((e = cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, device)) != cudaSuccess)
+        return bail(e, "SM count");
+    std::vector<int> order;
+    if (dispatch_order(g, nb, sm_count, order)) {
+        if ((e = cudaMalloc(&m->qorder, sizeof(int) * nb)) != cudaSuccess)
+            return bail(e, "qorder");
+        // synchronous copy from pageable memory: `order` is released on return
+        if ((e = cudaMemcpy(m->qorder, order.data(), sizeof(int) * nb, cudaMemcpyHostToDevice)) != cudaSuccess)
+            return bail(e, "qorder copy");
+    }
     // The scratch arrays are released by ~Scratch; cudaFree waits for the kernels.
     if ((e = cudaStreamSynchronize(cs)) != cudaSuccess)
         return bail(e, "mask build");
@@ -472,25 +514,18 @@ extern "C" void ra_mask_free(ra_mask* m)
     delete m;
 }
 
-// Device address of g_noalloc_scratch on the current device, looked up once per
-// device (host code cannot use the symbol itself as a device address).
+// Device address of g_noalloc_scratch in the current device's context.  Host
+// code cannot use the symbol itself as a device address.  The address is looked
+// up on every call (a cheap query) rather than cached per device ordinal: a
+// cached address would go stale if the device's primary context were reset and
+// the module loaded again.
 static ra_status noalloc_scratch_address(unsigned char** out)
 {
-    static std::mutex mu;
-    static unsigned char* addr[128] = {};
-    int dev = 0;
-    RA_CUDA_TRY(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= 128)
-        return fail(RA_ERR_UNSUPPORTED, "device ordinal %d is beyond the library's table", dev);
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "cudaGetSymbolAddress(builder scratch)");
-        addr[dev] = static_cast<unsigned char*>(p);
-    }
-    *out = addr[dev];
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetSymbolAddress(builder scratch)");
+    *out = static_cast<unsigned char*>(p);
     return RA_OK;
 }
 

@@ -84,14 +84,36 @@ struct WaitCtl {
     uint64_t timeout_ns;
 };
 
-static __device__ __noinline__ void report_timeout(const WaitCtl& w, int site)
+// Record a device error (the first one wins) and raise the CTA's abort flag.
+static __device__ __noinline__ void report_device_error(const WaitCtl& w, int status, int site)
 {
     *w.abort_flag = 1;
-    if (atomicCAS(w.err_word, 0, 5 /* RA_ERR_DEVICE_TIMEOUT */) == 0) {
+    if (atomicCAS(w.err_word, 0, status) == 0) {
         w.err_word[1] = site;
         w.err_word[2] = static_cast<int>(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
     }
 }
+
+static __device__ __forceinline__ void report_timeout(const WaitCtl& w, int site)
+{
+    report_device_error(w, 5 /* RA_ERR_DEVICE_TIMEOUT */, site);
+}
+
+// Bounds checks of the debug build (-DRA_DEBUG_BOUNDS): every global index and
+// TMA coordinate a kernel derives from its inputs is checked before use; a
+// failed check records RA_ERR_DEVICE_BOUNDS with its site, raises the abort
+// flag (the CTA's other roles leave their waits) and the caller skips the
+// access.  No trap, no fault.  The release build compiles the checks away.
+#ifdef RA_DEBUG_BOUNDS
+__device__ __forceinline__ bool in_bounds(const WaitCtl& w, bool ok, int site)
+{
+    if (!ok)
+        report_device_error(w, 6 /* RA_ERR_DEVICE_BOUNDS */, site);
+    return ok;
+}
+#else
+__device__ __forceinline__ bool in_bounds(const WaitCtl&, bool, int) { return true; }
+#endif
 
 // Wait for the phase with parity `parity` of `bar`.  False on timeout or when
 // another wait of this CTA (or another CTA) has already given up.
@@ -190,6 +212,16 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// Shift the 32-byte column group at taddr (lane aligned to 32) down by one TMEM
+// lane, asynchronously.  The PTX ISA lists MMA -> shift and shift -> MMA of the
+// same cta_group as pipelined pairs (executed in issue order), so a shift on a
+// column group that the next MMA overwrites orders that MMA after every earlier
+// MMA of the thread, whatever their accumulators.
+__device__ __forceinline__ void tmem_shift_down(uint32_t taddr)
+{
+    asm volatile("tcgen05.shift.cta_group::1.down [%0];" ::"r"(taddr) : "memory");
 }
 
 // Arrive once on `bar` when every tcgen05 operation issued so far by this thread completes.

@@ -156,8 +156,9 @@ extern "C" ra_status ra_swc_cache_step(ra_swc_cache* c, const void* Q_frame, con
     const int nk = held * c->s;
     const int* rp = c->row_ptr + static_cast<size_t>(held - 1) * (c->nbq + 1);
     const long long off = c->col_off[held - 1];
+    const int nnz = c->nbq * ((nk + TILE - 1) / TILE);  // every key tile of the held rows, per query tile
     ra_status st = attention_fwd_rect(Q_frame, c->K_ring, c->V_ring, O_frame, c->B, c->H, c->d, c->s, nk,
-                                      c->W * c->s, rp, c->col_idx + off, c->flag + off, c->nbq, scale, lse, cs);
+                                      c->W * c->s, rp, c->col_idx + off, c->flag + off, c->nbq, nnz, scale, lse, cs);
     if (st != RA_OK)
         return st;
     c->frames_seen += 1;

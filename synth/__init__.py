@@ -87,6 +87,20 @@ def normal_bf16(seed: int, tensor_id: int, shape, out: np.ndarray | None = None)
     return out.reshape(shape)
 
 
+def normal_bf16_heads(seed: int, tensor_id: int, shape, h0: int, h1: int) -> np.ndarray:
+    """Heads [h0, h1) of normal_bf16(seed, tensor_id, shape) for shape [B, H, n, d],
+    drawn directly from the counter-based stream (no other element is drawn)."""
+    B, H, n, d = shape
+    assert 0 <= h0 <= h1 <= H
+    out = np.empty((B, h1 - h0, n, d), dtype=np.uint16)
+    per_head = n * d
+    for b in range(B):
+        dst = out[b].reshape(-1)
+        _load().synth_normal(seed, tensor_id, (b * H + h0) * per_head, (h1 - h0) * per_head, None,
+                             dst.ctypes.data)
+    return out
+
+
 def normal_f32(seed: int, tensor_id: int, shape) -> np.ndarray:
     """The same stream as normal_bf16 before rounding (fp32)."""
     count = int(np.prod(shape))

@@ -66,3 +66,37 @@ def sampled_rows(seed, f, s, B, H, count=256):
 
 def scale_for(d):
     return 1.0 / math.sqrt(d)
+
+
+# ------------------------------------------------------------------ canaries
+# Output buffers of the GPU tests sit between two canary bands: a stray store
+# just before or after an output (a wrong row bound, a tail tile written past
+# n, a wrong head stride) changes a band, which check_canaries() reports.  The
+# band is 4096 elements (8 or 16 KB), so the output keeps 16-byte alignment.
+CANARY = 4096
+
+
+class Guarded:
+    """A CUDA tensor of `shape` and `dtype` (bf16 or fp32) inside canary bands."""
+
+    def __init__(self, shape, dtype, fill=float("nan")):
+        numel = int(np.prod(shape))
+        self.buf = torch.empty(numel + 2 * CANARY, dtype=dtype, device="cuda")
+        self.t = self.buf[CANARY:CANARY + numel].view(shape)
+        self.t.fill_(fill)
+        self._bits = torch.int16 if dtype == torch.bfloat16 else torch.int32
+        pattern = torch.arange(CANARY, dtype=torch.int64, device="cuda") * 40503 + 12345
+        mod = 1 << (16 if dtype == torch.bfloat16 else 32)
+        self._pattern = ((pattern % mod) - mod // 2).to(self._bits)
+        bits = self.buf.view(self._bits)
+        bits[:CANARY] = self._pattern
+        bits[-CANARY:] = self._pattern
+
+    def intact(self) -> bool:
+        bits = self.buf.view(self._bits)
+        return bool(torch.equal(bits[:CANARY], self._pattern) and torch.equal(bits[-CANARY:], self._pattern))
+
+
+def check_canaries(*guarded, what=""):
+    for i, g in enumerate(guarded):
+        assert g.intact(), f"{what}: a store landed outside output buffer {i}"

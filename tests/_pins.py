@@ -83,3 +83,58 @@ def block_mask_from_tiles(counts: np.ndarray, n: int) -> np.ndarray:
     """Element mask of block mode: every valid pair of every kept tile."""
     kept = counts > 0
     return np.kron(kept, np.ones((TILE, TILE), dtype=bool))[:n, :n]
+
+
+def radial_tile_stats_intervals(f: int, s: int):
+    """Tile statistics of eq. 4 at the 128 x 128 granularity, from the key
+    interval of each (query frame segment, key frame) pair instead of pairs.
+
+    Only for shapes where every frame distance keeps a diagonal band (w <= s for
+    D <= f - 1).  A query tile covers one or two frame segments of consecutive
+    positions [ka, kb]; in key frame j at distance D it keeps the positions
+    [ka - m, kb + m] (m = floor(s / w) - 1), so its kept key tiles are those that
+    interval touches.  A kept tile is FULL iff every (query segment, key segment)
+    pair inside it is within the band: max(kb - la, lb - ka) <= m for the key
+    segment [la, lb] of frame j, and the tile has no tail rows or keys.
+    Returns, per query tile, the sorted kept key tiles and the FULL ones."""
+    n = f * s
+    nb = -(-n // TILE)
+    assert 1 << (max(f - 1, 1).bit_length() - 1) <= s, "a frame distance with w > s"
+    m_of = np.empty(f, dtype=np.int64)
+    for D in range(f):
+        w = 1 << (max(D, 1).bit_length() - 1)
+        m_of[D] = s // w - 1
+    rows, fulls = [], []
+    frames = np.arange(f)
+    for qb in range(nb):
+        r0, r1 = qb * TILE, min(n, qb * TILE + TILE) - 1
+        segs = [(i, max(r0, i * s) - i * s, min(r1, i * s + s - 1) - i * s) for i in range(r0 // s, r1 // s + 1)]
+        kept = set()
+        for i, ka, kbp in segs:
+            m = m_of[np.abs(i - frames)]
+            lo = np.maximum(0, ka - m) + frames * s
+            hi = np.minimum(s - 1, kbp + m) + frames * s
+            for a, b in zip(lo // TILE, hi // TILE):
+                kept.update(range(int(a), int(b) + 1))
+        kept = np.array(sorted(kept), dtype=np.int64)
+        rows.append(kept)
+        full = []
+        fulls.append(full)
+        if r1 - r0 + 1 < TILE:
+            continue
+        for kb in kept:
+            c0, c1 = kb * TILE, min(n, kb * TILE + TILE) - 1
+            if c1 - c0 + 1 < TILE:
+                continue
+            ok = True
+            for i, ka, kbp in segs:
+                for j in range(c0 // s, c1 // s + 1):
+                    la, lb = max(c0, j * s) - j * s, min(c1, j * s + s - 1) - j * s
+                    if max(kbp - la, lb - ka) > m_of[abs(i - j)]:
+                        ok = False
+                        break
+                if not ok:
+                    break
+            if ok:
+                full.append(int(kb))
+    return rows, fulls

@@ -115,6 +115,13 @@ def test_backward_rejects_bad_arguments(ra):
     assert call(d=256) == ra.RA_ERR_UNSUPPORTED
     assert call(mode=3) == ra.RA_ERR_INVALID_ARG
     assert call(scale=-1.0) == ra.RA_ERR_INVALID_ARG
+    # an output aliasing an input or another output (dQ is written before the
+    # dK / dV kernel reads Q and dO)
+    for out_name in ("dQ", "dK", "dV", "ws"):
+        for other in ("Q", "K", "V", "O", "dO", "lse", "dQ", "dK", "dV", "ws"):
+            if other != out_name:
+                assert call(**{out_name: args[other]}) == ra.RA_ERR_INVALID_ARG, (out_name, other)
+                assert b"alias" in ra.ra_last_error()
 
 
 def test_swc_cache_rejects_bad_arguments(ra):
@@ -130,6 +137,15 @@ def test_swc_cache_rejects_bad_arguments(ra):
     assert ra.ra_swc_cache_reset(None) == ra.RA_ERR_INVALID_ARG
     assert ra.ra_swc_cache_copy_rings_to_host(None, None, None) == ra.RA_ERR_INVALID_ARG
     ra.ra_swc_cache_free(None)
+
+
+def test_release_library_has_no_bounds_checks(ra):
+    """The bounds self-test needs the debug variant; the release build says so
+    without touching the GPU."""
+    if ra.VARIANT == "release":
+        assert ra.ra_selftest_bounds(None) == ra.RA_ERR_UNSUPPORTED
+        assert b"RA_DEBUG_BOUNDS" in ra.ra_last_error()
+    assert ra.ra_status_string(ra.RA_ERR_DEVICE_BOUNDS) == b"device bounds check failed"
 
 
 def test_timeout_settings_are_range_checked(ra):

@@ -45,8 +45,13 @@ def _fwd_bwd(spec, Qh, Kh, Vh, dOh, mode):
     lse = torch.empty((B, H, n), dtype=torch.float32, device="cuda")
     scale = _gpu.scale_for(d)
     o = ra.attention_fwd(q, k, v, m, scale=scale, mode=mode, lse=lse)
-    dq, dk, dv = ra.attention_bwd(q, k, v, o, do, lse, m, scale=scale, mode=mode)
+    # gradients and the D workspace inside canary bands (no store outside them)
+    g = [_gpu.Guarded((B, H, n, d), torch.bfloat16) for _ in range(3)]
+    g_ws = _gpu.Guarded((B, H, n), torch.float32)
+    dq, dk, dv = ra.attention_bwd(q, k, v, o, do, lse, m, scale=scale, mode=mode, dq=g[0].t, dk=g[1].t,
+                                  dv=g[2].t, workspace=g_ws.t)
     assert ra.device_status() == ra.RA_OK
+    _gpu.check_canaries(*g, g_ws, what=f"backward {spec} {mode}")
     return dq, dk, dv, m
 
 
@@ -139,37 +144,80 @@ def _full_inputs(name):
     return c, Qh, Kh, Vh, synth.dout_bf16(name)
 
 
+# Relative rounding error of one bf16 rounding (8-bit significand, round to
+# nearest even): at most 2^-8 in magnitude and uniform over the spacing, so its
+# standard deviation is at most 2^-8 / sqrt(3) (attained at the bottom of a binade).
+EPS_BF16 = 2.0 ** -8 / np.sqrt(3.0)
+
+
 @pytest.mark.parametrize("name,mask_i", [("hunyuan108k", 0), ("wan_radial", 0), ("wan_radial", 1)],
                          ids=lambda x: str(x))
 def test_full_size_sampled_query_rows_and_sums(orc, name, mask_i):
-    """Full size, all heads, in the benchmark's launch configuration (block mode):
-    dQ on 256 // H + 8 seeded rows per head (boundary rows included) against the
-    oracle one row at a time, and at
-    every head and column the identity that holds at any size
-        sum_j dV_j = sum_i dO_i   (rows of P sum to 1).
-    Its bound is 8 standard deviations of three roundings: dV to bf16 and the P
-    operand to bf16 (2^-9 / sqrt(3) of ||dV|| each), and the fp32 row sums of the
-    forward that normalise P (a random walk over the k computed keys of a row,
-    2^-23 sqrt(k) per row, times ||dO||)."""
+    """Full size, all heads, in the benchmark's launch configuration (block mode).
+
+    dQ on the same 256 seeded rows in every head (boundary rows included) against
+    the oracle one row at a time; and, at every head and column, two identities
+    that hold at any size, each within 8 standard deviations of the roundings
+    that can break it:
+
+      sum_j dV_j = sum_i dO_i, because the rows of P sum to 1.  Roundings: dV to
+        bf16 and the P operand to bf16 (EPS_BF16 ||dV|| each), and the fp32 row
+        sums that normalise P (a random walk over the k computed keys of a row,
+        2^-23 sqrt(k) per row, times ||dO||).
+
+      sum_j dK_j = 0, because sum_j dS_ij = sum_j P_ij dP_ij - D_i sum_j P_ij and
+        sum_j P_ij dP_ij = <dO_i, O_i> = D_i.  The kernel takes D_i from the
+        forward's bf16 O, so row i leaves eps_i = <dO_i, O_i - O_fwd_i>, and
+        sum_j dK_jc = scale sum_i eps_i Q_ic: a random sum of standard deviation
+        scale rms(eps) ||Q_c||, with rms(eps) measured on the sampled rows
+        against the oracle's exact O.  Roundings: dK to bf16 and the dS operand
+        to bf16 (EPS_BF16 ||dK_c|| each, since dK = scale dS^T Q with unit-variance
+        Q gives ||dK_c|| = scale ||dS||_F)."""
     _gpu.need_gpu()
     c, Qh, Kh, Vh, dOh = _full_inputs(name)
     spec = oracle.spec_from(c["masks"][mask_i], c["f"], c["s"], c["grid"])
-    dq, dk, dv, m = _fwd_bwd(spec, Qh, Kh, Vh, dOh, "block")
-    B, H, n, d = Qh.shape
-    row_bh, row_q = _gpu.sampled_rows(synth.config_seed(name), c["f"], c["s"], B, H, count=256 // H + 8)
-    want = orc.attention_bwd_query_rows(Qh, Kh, Vh, dOh, spec, oracle.BLOCK, _gpu.scale_for(d), row_bh, row_q)
+    ra = _gpu.ra()
+    m = _gpu_mask(spec)
+    q, k, v, do = (_gpu.to_device(t) for t in (Qh, Kh, Vh, dOh))
+    B, H, n, d = q.shape
+    scale = _gpu.scale_for(d)
+    lse = torch.empty((B, H, n), dtype=torch.float32, device="cuda")
+    o = ra.attention_fwd(q, k, v, m, scale=scale, mode="block", lse=lse)
+    dq, dk, dv = ra.attention_bwd(q, k, v, o, do, lse, m, scale=scale, mode="block")
+    assert ra.device_status() == ra.RA_OK
+
+    row_bh, row_q = _gpu.sampled_rows(synth.config_seed(name), c["f"], c["s"], B, H, count=256)
+    want = orc.attention_bwd_query_rows(Qh, Kh, Vh, dOh, spec, oracle.BLOCK, scale, row_bh, row_q)
     got = _gpu.gather_rows(_gpu.to_f64(dq), row_bh, row_q)
     assert_grad_close(got, want, f"{name} dQ sampled")
-    dv_sum = dv.double().sum(dim=2).cpu().numpy()
-    dv_norm = np.sqrt((dv.double() ** 2).sum(dim=2).cpu().numpy())
-    dO64 = synth.bf16_bits_to_f32(dOh).astype(np.float64)
-    dO_sum, dO_norm = dO64.sum(axis=2), np.sqrt((dO64 ** 2).sum(axis=2))
+
     keys_per_row = m.info["block_pairs"] / n
-    eps_b = 2.0 ** -9 / np.sqrt(3.0)
+
+    def sum_and_norm(t):  # over the rows of each (b, h), per column, in fp64 on the device
+        t64 = t.double()
+        out = t64.sum(dim=2).cpu().numpy(), torch.sqrt((t64 ** 2).sum(dim=2)).cpu().numpy()
+        del t64
+        return out
+
+    # sum_j dV_j = sum_i dO_i
+    dv_sum, dv_norm = sum_and_norm(dv)
+    dO_sum, dO_norm = sum_and_norm(do)
     eps_n = 2.0 ** -23 * np.sqrt(keys_per_row)
-    sigma = np.sqrt(2.0 * (eps_b * dv_norm) ** 2 + (eps_n * dO_norm) ** 2)
+    sigma = np.sqrt(2.0 * (EPS_BF16 * dv_norm) ** 2 + (eps_n * dO_norm) ** 2)
     err = np.abs(dv_sum - dO_sum)
     assert np.all(err <= 8 * sigma), f"sum_j dV_j != sum_i dO_i: worst {float(np.max(err / sigma)):.1f} sigma"
+
+    # sum_j dK_j = 0
+    o_exact, _, _ = orc.attention_rows(Qh, Kh, Vh, spec, oracle.BLOCK, scale, row_bh, row_q)
+    o_fwd = _gpu.gather_rows(_gpu.to_f64(o), row_bh, row_q)
+    dO_rows = synth.bf16_bits_to_f32(dOh.reshape(B * H, n, d)[row_bh, row_q]).astype(np.float64)
+    eps = np.sum(dO_rows * (o_exact - o_fwd), axis=1)                      # one per sampled row
+    rms_eps = np.sqrt(np.bincount(row_bh, eps ** 2, B * H) / np.bincount(row_bh, None, B * H))
+    dk_sum, dk_norm = (x.reshape(B * H, d) for x in sum_and_norm(dk))
+    q_norm = sum_and_norm(q)[1].reshape(B * H, d)
+    sigma_k = np.sqrt(2.0 * (EPS_BF16 * dk_norm) ** 2 + (scale * rms_eps[:, None] * q_norm) ** 2)
+    ratio = np.abs(dk_sum) / sigma_k
+    assert np.all(ratio <= 8), f"sum_j dK_j != 0: worst {float(np.max(ratio)):.1f} sigma"
 
 
 def _key_rows_check(orc, name, mask_i, H, keys, what):

@@ -26,9 +26,18 @@ def _run(spec: oracle.MaskSpec, Qh, Kh, Vh, mode: str, lse=False):
                 spec.sink_tokens)
     q, k, v = (_gpu.to_device(t) for t in (Qh, Kh, Vh))
     B, H, n, d = q.shape
-    out_lse = torch.empty((B, H, n), dtype=torch.float32, device="cuda") if lse else None
-    o = ra.attention_fwd(q, k, v, m, scale=_gpu.scale_for(d), mode=mode, lse=out_lse)
+    # NaN-filled outputs inside canary bands: every row must be written, whichever
+    # CTA the mask's dispatch order gives its query tile to, and nothing else
+    g_o = _gpu.Guarded((B, H, n, d), torch.bfloat16)
+    g_lse = _gpu.Guarded((B, H, n), torch.float32) if lse else None
+    out_lse = g_lse.t if lse else None
+    o = g_o.t
+    ra.attention_fwd(q, k, v, m, scale=_gpu.scale_for(d), mode=mode, lse=out_lse, out=o)
     assert ra.device_status() == ra.RA_OK
+    _gpu.check_canaries(*([g_o, g_lse] if lse else [g_o]), what=f"forward {spec} {mode}")
+    assert bool(torch.isfinite(o).all()), "an output row was not written"
+    if lse:
+        assert not bool(torch.isnan(out_lse).any()), "an lse entry was not written"
     return o, out_lse, m
 
 

@@ -67,6 +67,57 @@ def test_radial_bound_large_shapes_closed_form():
         assert _pins.radial_closed_form_total(f, s) <= 4 * s * s * f * int(math.floor(math.log2(f)))
 
 
+# Totals of eq. 4 on the three large radial shapes, per head (Radial Attention,
+# eq. 4 at the 128 x 128 tiles of sec. 6): kept pairs, kept tiles, FULL tiles,
+# fewest and most kept tiles in a query-tile row.
+LARGE_RADIAL = {
+    (41, 1560): (1322566560, 117526, 48791, 140, 268),      # Wan-shaped
+    (30, 3600): (4547300400, 321300, 233963, 212, 464),     # HunyuanVideo-shaped, 108000 tokens
+    (128, 3600): (31997441936, 2818574, 1251414, 466, 880),  # 4x long, 460800 tokens
+}
+
+
+@pytest.mark.parametrize("f,s", sorted(LARGE_RADIAL))
+def test_radial_large_shape_literal_totals(f, s):
+    """The literal totals from the band closed form (kept pairs) and from the
+    per-frame-pair interval enumeration (tiles)."""
+    kept, nnz, full, rmin, rmax = LARGE_RADIAL[(f, s)]
+    assert _pins.radial_closed_form_total(f, s) == kept
+    rows, fulls = _pins.radial_tile_stats_intervals(f, s)
+    lengths = [len(r) for r in rows]
+    assert (sum(lengths), sum(map(len, fulls)), min(lengths), max(lengths)) == (nnz, full, rmin, rmax)
+
+
+def test_radial_wan_oracle_tiles_equal_literal_totals(orc):
+    """The oracle's brute-force tile counts of the whole Wan-shaped mask: the
+    literal totals, and the interval enumeration's kept and FULL tiles row by row."""
+    f, s = 41, 1560
+    kept, nnz, full, rmin, rmax = LARGE_RADIAL[(f, s)]
+    counts = orc.tile_counts(MaskSpec(RADIAL, f, s))
+    per_row = (counts > 0).sum(axis=1)
+    assert (int(counts.sum()), int((counts > 0).sum()), int((counts == 128 * 128).sum())) == (kept, nnz, full)
+    assert (int(per_row.min()), int(per_row.max())) == (rmin, rmax)
+    rows, fulls = _pins.radial_tile_stats_intervals(f, s)
+    for qb in range(counts.shape[0]):
+        assert np.array_equal(np.flatnonzero(counts[qb] > 0), rows[qb]), qb
+        assert np.array_equal(np.flatnonzero(counts[qb] == 128 * 128), fulls[qb]), qb
+
+
+def test_radial_long_oracle_tiles_equal_intervals_on_sampled_rows(orc):
+    """460800 tokens: the oracle's brute-force tile counts of 16 query tiles
+    (first, last, frame boundaries, seeded) equal the interval enumeration whose
+    totals are pinned above."""
+    f, s = 128, 3600
+    nb = f * s // 128
+    rng = np.random.default_rng(460800)
+    qbs = np.unique(np.r_[0, nb - 1, 28, 29, 1799, 1800, rng.integers(0, nb, 10)]).astype(np.int32)
+    counts = orc.tile_counts(MaskSpec(RADIAL, f, s), qbs)
+    rows, fulls = _pins.radial_tile_stats_intervals(f, s)
+    for r, qb in enumerate(qbs):
+        assert np.array_equal(np.flatnonzero(counts[r] > 0), rows[qb]), qb
+        assert np.array_equal(np.flatnonzero(counts[r] == 128 * 128), fulls[qb]), qb
+
+
 # ------------------------------------------------------------ other families
 
 def test_window3d_counts_printed_on_tutorial(orc):

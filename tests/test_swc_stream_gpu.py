@@ -25,10 +25,14 @@ def _stream(Qh, Kh, Vh, s, W, frames=None):
     outs, lses = [], []
     for i in range(f):
         sl = slice(i * s, (i + 1) * s)
-        lse = torch.empty((B, H, s), dtype=torch.float32, device="cuda")
-        o = cache.step(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(), v[:, :, sl].contiguous(), lse=lse)
+        # the step's outputs inside canary bands: no store outside them
+        g_o, g_lse = _gpu.Guarded((B, H, s, d), torch.bfloat16), _gpu.Guarded((B, H, s), torch.float32)
+        o = cache.step(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(), v[:, :, sl].contiguous(), out=g_o.t,
+                       lse=g_lse.t)
+        _gpu.check_canaries(g_o, g_lse, what=f"SWC step {i}")
+        assert bool(torch.isfinite(o).all()), f"SWC step {i}: an output row was not written"
         outs.append(_gpu.to_f64(o))
-        lses.append(lse.cpu().numpy().astype(np.float64))
+        lses.append(g_lse.t.cpu().numpy().astype(np.float64))
     assert ra.device_status() == ra.RA_OK
     return outs, lses, cache
 

@@ -114,3 +114,12 @@ def test_sampled_rows_hold_the_boundary_rows(f, s):
     assert need <= set(rows.tolist())
     np.testing.assert_array_equal(rows, synth.sample_rows(1234, f, s))
     assert not np.array_equal(rows, synth.sample_rows(1235, f, s)) or n <= 256
+
+
+def test_head_slices_equal_the_full_tensor():
+    """A rank's heads drawn on their own are the same elements as the slice of the
+    whole tensor (B > 1, uneven ranges, empty range)."""
+    shape = (2, 5, 37, 16)
+    full = synth.normal_bf16(1234, 2, shape)
+    for h0, h1 in [(0, 5), (0, 2), (2, 5), (3, 4), (4, 4)]:
+        assert np.array_equal(synth.normal_bf16_heads(1234, 2, shape, h0, h1), full[:, h0:h1])

@@ -23,13 +23,16 @@ CASES = [
     ("radial", 30, 700, dict()),                                   # n = 21000, ragged tail
     ("window3d", 9, 99, dict(grid_h=9, grid_w=11, r_t=2, r_s=4)),  # n = 891
     ("swc", 41, 1560, dict(window_frames=16)),                     # n = 63960
+    ("radial", 32, 4096, dict()),                                  # n = 131072: nb = 1024, the whole scratch
+    ("window3d", 31, 4225, dict(grid_h=65, grid_w=65, r_t=1, r_s=3, sink_tokens=300)),  # nb = 1024, ragged tail
+    ("radial", 30, 700, dict(sink_tokens=700)),                    # the first frame global
     ("radial", 30, 700, dict()),                                   # the first mask again
 ]
 
 
 def _params(ra, kw):
     return ra.ra_mask_params(kw.get("grid_h", 0), kw.get("grid_w", 0), kw.get("r_t", 0), kw.get("r_s", 0),
-                             kw.get("window_frames", 0))
+                             kw.get("window_frames", 0), kw.get("sink_tokens", 0))
 
 
 def _noalloc(ra, family, f, s, kw, capacity):
@@ -55,7 +58,7 @@ def test_noalloc_matches_the_allocating_builder_on_consecutive_calls():
     ra = _gpu.ra()
     for family, f, s, kw in CASES:
         ref_mask = ra.Mask(family, f, s, kw.get("grid_h", 0), kw.get("grid_w", 0), kw.get("r_t", 0),
-                           kw.get("r_s", 0), kw.get("window_frames", 0))
+                           kw.get("r_s", 0), kw.get("window_frames", 0), kw.get("sink_tokens", 0))
         ref = ref_mask.to_host()
         st, got, info = _noalloc(ra, family, f, s, kw, capacity=ref["nnz"])
         assert st == ra.RA_OK, ra.ra_last_error()
