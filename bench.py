@@ -259,6 +259,14 @@ def time_two_streams(step, n_steps, main_stream):
     return e0.elapsed_time(e1)
 
 
+def fwd_kernel_name(info, c, mode):
+    """The forward kernel instance the library runs for this mask and mode: rows
+    averaging fewer than 4096 computed keys keep P as hi + lo (SPLIT_P)."""
+    n = c["f"] * c["s"]
+    pairs = info["block_pairs"] if mode == "block" else info["kept_pairs"]
+    return f"attn_fwd_kernel<{c['d']}, {'true' if pairs < 4096 * n else 'false'}>"
+
+
 def flops_per_call(info, c, mode, kind="fwd"):
     pairs = info["block_pairs"] if mode == "block" else info["kept_pairs"]
     return (4.0 if kind == "fwd" else 10.0) * c["d"] * pairs * c["B"] * c["H"]
@@ -768,7 +776,7 @@ def main():
                 "traffic": recorded_traffic(args.workload, args.mode, mask["family"], args.pass_),
                 "peak_source": f"{peak_src} bf16 {'burst' if timed_alone else 'sustained'} (MEASURED_PEAKS.json)"
                 if peak_src == "measured" else "fallback 1.59 PFLOP/s burst / 1.4 sustained",
-                "kernel": ("attn_fwd_kernel<%d>" % d) if not bwd else
+                "kernel": fwd_kernel_name(info, c, args.mode) if not bwd else
                 ("ra_attention_bwd call: bwd_dot_kernel<%d> + bwd_dq_kernel<%d> + bwd_dkdv_kernel<%d>" % (d, d, d)),
                 "flop_per_launch": flop,
                 "flop_executed_per_launch": flops_per_call(info, c_rank, "block", args.pass_),

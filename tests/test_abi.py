@@ -148,6 +148,13 @@ def test_release_library_has_no_bounds_checks(ra):
     assert ra.ra_status_string(ra.RA_ERR_DEVICE_BOUNDS) == b"device bounds check failed"
 
 
+def test_kernel_settings_are_range_checked(ra):
+    assert ra.ra_set_pv_precision(7) == ra.RA_ERR_INVALID_ARG
+    assert ra.ra_set_pv_precision(-1) == ra.RA_ERR_INVALID_ARG
+    for v in (ra.RA_PV_BF16, ra.RA_PV_SPLIT, ra.RA_PV_AUTO):
+        assert ra.ra_set_pv_precision(v) == ra.RA_OK
+
+
 def test_timeout_settings_are_range_checked(ra):
     assert ra.ra_set_wait_timeout_ns(10) == ra.RA_ERR_INVALID_ARG
     assert ra.ra_set_wait_timeout_ns(4_000_000_000) == ra.RA_OK

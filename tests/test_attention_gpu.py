@@ -152,6 +152,22 @@ def test_deterministic_bits():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+def test_deterministic_bits_bf16p():
+    """The same bits on repeated calls with bf16 P at d = 128 (the large
+    workloads' path), a ragged tail and token-exact partial tiles."""
+    _gpu.need_gpu()
+    ra = _gpu.ra()
+    ra.check(ra.ra_set_pv_precision(ra.RA_PV_BF16), "ra_set_pv_precision")
+    try:
+        spec = oracle.MaskSpec(oracle.RADIAL, 13, 300)
+        Q, K, V = (synth.normal_bf16(55, t, (1, 3, spec.n, 128)) for t in range(3))
+        a, _, _ = _run(spec, Q, K, V, "token_exact")
+        b, _, _ = _run(spec, Q, K, V, "token_exact")
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    finally:
+        ra.ra_set_pv_precision(ra.RA_PV_AUTO)
+
+
 def test_host_io_entry_point_matches_device_call():
     _gpu.need_gpu()
     ra = _gpu.ra()

@@ -98,3 +98,14 @@ def test_reference_arm_line(args):
     assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert _reference_line(args, rank="1") is None
+
+
+def test_forward_kernel_name_follows_the_library_choice(bench):
+    """Rows of >= 4096 computed keys on average keep bf16 P; fewer keep hi + lo P."""
+    import synth
+    big = synth.CONFIGS["hunyuan108k"]
+    info = {"block_pairs": 321300 * 128 * 128, "kept_pairs": 4547300400}
+    assert bench.fwd_kernel_name(info, big, "block") == "attn_fwd_kernel<128, false>"
+    tiny = synth.CONFIGS["tiny_radial"]
+    assert bench.fwd_kernel_name({"block_pairs": 512 * 512, "kept_pairs": 191872}, tiny, "token_exact") == \
+        "attn_fwd_kernel<64, true>"
