@@ -780,7 +780,16 @@ def main():
                 ("ra_attention_bwd call: bwd_dot_kernel<%d> + bwd_dq_kernel<%d> + bwd_dkdv_kernel<%d>" % (d, d, d)),
                 "flop_per_launch": flop,
                 "flop_executed_per_launch": flops_per_call(info, c_rank, "block", args.pass_),
-                "algorithmic_bytes_per_launch": bytes_qkvo}
+                "algorithmic_bytes_per_launch": bytes_qkvo,
+                "algorithmic_gbs": bytes_qkvo / avg_launch_s / 1e9}
+    if roofline["traffic"] is not None:
+        # the recorded DRAM bytes are per launch over all heads of the workload as
+        # configured; heads are independent, so a launch over fewer scales with them
+        base = synth.CONFIGS[args.workload]
+        traffic = roofline["traffic"] * (c_rank["B"] * c_rank["H"]) / (base["B"] * base["H"])
+        roofline["traffic"] = traffic
+        roofline["dram_gbs"] = traffic / avg_launch_s / 1e9
+        roofline["dram_frac_of_hbm"] = roofline["dram_gbs"] / hbm
 
     # ---- end to end: host buffers through the C ABI (H2D + kernel + D2H per step)
     e2e = None
@@ -870,6 +879,13 @@ def main():
         cpu = {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
         cpu.update(cpu_oracle_extras(args.workload, mask, args.mode, c, kind=args.pass_))
 
+    # the fraction of what the tensor pipe can do at the clock the run actually
+    # had: 148 SMs x 8192 dense bf16 FLOP per clock x the median sampled SM clock
+    clk = clk.summary()
+    if clk.get("sm_mhz"):
+        clock_peak = 148 * 8192 * clk["sm_mhz"] * 1e6 / 1e12
+        roofline["clock_peak_tflops"] = clock_peak
+        roofline["frac_of_clock_peak"] = achieved / clock_peak
     tile_total = info["nb"] ** 2
     line = {
         "metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -900,7 +916,7 @@ def main():
         "mask_build_ms": mask_build_ms,
         "pct_of_peak": 100.0 * roofline["frac"],
         "roofline": roofline,
-        "clocks": clk.summary(),
+        "clocks": clk,
         "gpu_launches": args.steps * launches_per_step,
         "e2e": e2e,
         "cpu_baseline": cpu,

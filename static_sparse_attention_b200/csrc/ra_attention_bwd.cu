@@ -47,6 +47,7 @@ struct BwdParams {
     const int* ptr;            // row_ptr (dQ pass) or col_ptr (dK/dV pass)
     const int* idx;            // col_idx or row_idx
     const unsigned char* flag; // flag or tflag
+    const int* order;          // tile of CTA x (the mask's dispatch order), or null for x itself
     int nnz;                   // entries of idx / flag (bounds checks of the debug build)
     const float* lse;          // [B*H, n] natural log
     const float* Dv;           // [B*H, n] rowsum(dO * O)
@@ -215,7 +216,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::BAR_OFF + 8 * BB::COUNT + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int qb = p.order ? p.order[blockIdx.x] : static_cast<int>(blockIdx.x);
+    const int h = blockIdx.y, b = blockIdx.z;
     const int bh = b * p.H + h;
     const int n = p.g.n;
     WaitCtl wc{abort_flag, p.err, p.timeout_ns};
@@ -228,8 +230,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
         }
         fence_barrier_init();
         fence_proxy_async_smem();
-        // (debug build) this tile's CSR row is in range
-        if (!*abort_flag)
+        // (debug build) this CTA's tile and its CSR row are in range
+        if (!*abort_flag && in_bounds(wc, qb >= 0 && qb < p.nb, BSITE_B_TILE))
             in_bounds(wc, 0 <= p.ptr[qb] && p.ptr[qb] <= p.ptr[qb + 1] && p.ptr[qb + 1] <= p.nnz, BSITE_B_ROW);
     }
     if (warp == DQ_MMA_WARP) {
@@ -560,7 +562,8 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
     float* st_d = st_l2 + TILE;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int kb = p.order ? p.order[blockIdx.x] : static_cast<int>(blockIdx.x);
+    const int h = blockIdx.y, b = blockIdx.z;
     const int bh = b * p.H + h;
     const int n = p.g.n;
     WaitCtl wc{abort_flag, p.err, p.timeout_ns};
@@ -573,8 +576,8 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
         }
         fence_barrier_init();
         fence_proxy_async_smem();
-        // (debug build) this tile's CSR row is in range
-        if (!*abort_flag)
+        // (debug build) this CTA's tile and its CSR row are in range
+        if (!*abort_flag && in_bounds(wc, kb >= 0 && kb < p.nb, BSITE_B_TILE))
             in_bounds(wc, 0 <= p.ptr[kb] && p.ptr[kb] <= p.ptr[kb + 1] && p.ptr[kb + 1] <= p.nnz, BSITE_B_ROW);
     }
     if (warp == KV_MMA_WARP) {
@@ -980,6 +983,10 @@ ra_status run_bwd(const void* Q, const void* K, const void* V, const void* O, co
     p.H = H;
     p.mode = mode;
     p.nnz = static_cast<int>(m->nnz);
+    // Query tiles (dQ pass) and key tiles (dK / dV pass) in the mask's dispatch
+    // order: by in-frame position band, then frame, so that the CTAs resident
+    // together walk overlapping tiles (eq. 4 is symmetric in query and key).
+    p.order = m->qorder;
     p.lse = lse;
     p.Dv = Dws;
     p.scale = scale;
