@@ -24,8 +24,9 @@ struct ra_mask {
     int* col_ptr;
     int* row_idx;
     unsigned char* tflag;
-    // Dispatch order of the forward's query tiles (CTA x runs query tile
-    // qorder[x]); null when it is the identity.
+    // Dispatch order of the attention kernels' tiles: CTA x of the forward and
+    // of the dQ pass runs query tile qorder[x], CTA x of the dK / dV pass key
+    // tile qorder[x]; null when it is the identity.
     int* qorder;
 };
 

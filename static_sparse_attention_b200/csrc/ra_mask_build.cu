@@ -249,8 +249,9 @@ __global__ void __launch_bounds__(128) col_compact_kernel(const int* __restrict_
     }
 }
 
-// The order in which the forward's CTAs take query tiles: sorted by in-frame
-// position band, then by frame.  eq. 4 keeps, in every key frame, a band of
+// The order in which the attention kernels' CTAs take their tiles (query tiles
+// of the forward and the dQ pass, key tiles of the dK / dV pass, by the mask's
+// symmetry in query and key): sorted by in-frame position band, then by frame.  eq. 4 keeps, in every key frame, a band of
 // positions centred on the query's own in-frame position, so query tiles of one
 // position band over many frames read overlapping key tiles; with the query
 // tiles of a head in plain order the resident CTAs instead cover a few whole
