@@ -111,6 +111,15 @@ def sources_sha256(kind="fwd"):
     return h.hexdigest()[:16]
 
 
+def mask_key(mask: dict) -> str:
+    """The mask part of a traffic record's key: the family, and the number of
+    global (sink) tokens when there are any (they change the tiles walked)."""
+    key = mask["family"]
+    if mask.get("sink_tokens"):
+        key += f"+sink{mask['sink_tokens']}"
+    return key
+
+
 def recorded_traffic(workload, mode, mask_family, kind="fwd"):
     """DRAM bytes per launch (per call, for the backward's kernels together) from
     the committed ncu summary, if it was taken on the current kernel sources
@@ -773,7 +782,7 @@ def main():
     peak = burst if timed_alone else sustained
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak,
-                "traffic": recorded_traffic(args.workload, args.mode, mask["family"], args.pass_),
+                "traffic": recorded_traffic(args.workload, args.mode, mask_key(mask), args.pass_),
                 "peak_source": f"{peak_src} bf16 {'burst' if timed_alone else 'sustained'} (MEASURED_PEAKS.json)"
                 if peak_src == "measured" else "fallback 1.59 PFLOP/s burst / 1.4 sustained",
                 "kernel": fwd_kernel_name(info, c, args.mode) if not bwd else

@@ -109,3 +109,11 @@ def test_forward_kernel_name_follows_the_library_choice(bench):
     tiny = synth.CONFIGS["tiny_radial"]
     assert bench.fwd_kernel_name({"block_pairs": 512 * 512, "kept_pairs": 191872}, tiny, "token_exact") == \
         "attn_fwd_kernel<64, true>"
+
+
+def test_traffic_record_key_tells_sink_masks_apart(bench):
+    """A mask with global tokens walks other tiles: it does not take the record of
+    the plain mask of the same family."""
+    assert bench.mask_key({"family": "radial"}) == "radial"
+    assert bench.mask_key({"family": "radial", "sink_tokens": 3600}) == "radial+sink3600"
+    assert bench.recorded_traffic("hunyuan108k", "block", "radial+sink3600") is None
