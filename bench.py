@@ -564,7 +564,8 @@ def run_stream(args, c, mask, world, rank, dev):
             "parallelism": f"{world} independent streams (one per GPU), no collective",
         },
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak,
+                     "traffic": recorded_traffic(args.workload, "exact", f"swc{W}-stream", "fwd"),
                      "peak_source": f"{peak_src} bf16 {'burst' if total_ms < 1000.0 else 'sustained'}",
                      "kernel": "attn_fwd_kernel<%d> over the ring (plus two 2D copies of the frame's K, V)" % d,
                      "flop_per_launch": flop},
@@ -637,12 +638,52 @@ def run_policy(args, c, mask, world, rank, dev):
     if ra.device_status() != ra.RA_OK:
         raise SystemExit("device status error after the timed region")
     total_ms = max_over_ranks(t0.elapsed_time(t1), world, f"cuda:{dev}")
+
+    # ---- end to end: two denoising steps of the schedule (the first, dense warm-up
+    # step and the last one) through ra_attention_fwd_host, every call copying its
+    # Q, K, V in from pinned host memory and its O out; consecutive calls on two
+    # streams with their own staging buffers
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).pin_memory() for h in host)
+        ho = [torch.empty(shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        dev_sets = [(q, k, v, o), tuple(torch.empty_like(q) for _ in range(4))]
+        e_calls = [policy.mask(t, l) for t in sorted({0, T - 1}) for l in range(L)]
+        e_flop = sum(f_dense if m is dense else f_sparse for m in e_calls)
+
+        def e2e_call(i, st):
+            m = e_calls[i % len(e_calls)]
+            dq_, dk_, dv_, do_ = dev_sets[i % 2]
+            ra.attention_fwd_host(hq, hk, hv, ho[i % 2], dq_, dk_, dv_, do_, m, scale=scale,
+                                  mode=args.mode if m is sparse else "block", stream=st)
+
+        time_two_streams(e2e_call, 2, stream)  # warm-up
+        if world > 1:
+            dist.barrier()
+        e_ms = max_over_ranks(time_two_streams(e2e_call, len(e_calls), stream), world, f"cuda:{dev}")
+        e2e = {"value": e_flop * world / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms / 2, "h2d_bytes_per_step": 3 * q.numel() * 2 * L,
+               "d2h_bytes_per_step": o.numel() * 2 * L,
+               "path": "two denoising steps of the schedule (the first and the last), every call through "
+                       "ra_attention_fwd_host (pinned host Q,K,V -> device, kernel, device -> pinned host O), "
+                       "consecutive calls on two streams with their own staging buffers"}
+        del hq, hk, hv, ho, dev_sets
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
     calls = T * L
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        # the oracle on bounded samples of both masks, combined with the schedule's
+        # mix of calls: the time the schedule's FLOP would take at those rates
+        v_s, threads, desc_s = cpu_oracle_sample(args.workload, mask, args.mode, c, target_s=8.0)
+        v_d, _, desc_d = cpu_oracle_sample(args.workload, dict(family="dense"), "block", c, target_s=8.0)
+        cpu_s = (calls - n_dense) * f_sparse / (v_s * 1e12) + n_dense * f_dense / (v_d * 1e12)
+        cpu = {"value": flop / cpu_s / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{mask['family']} mask: {desc_s}; dense mask: {desc_d}; combined by the schedule's "
+                         f"{calls - n_dense} {mask['family']} and {n_dense} dense calls"}
     all_dense_ms = calls * per_call["dense"]
     burst, sustained, _, peak_src = measured_peaks()
     achieved = flop / (total_ms / 1e3) / 1e12
@@ -666,8 +707,8 @@ def run_policy(args, c, mask, world, rank, dev):
                      "kernel": "attn_fwd_kernel<%d> (sparse and dense calls)" % d, "flop_per_launch": flop / calls},
         "clocks": clk.summary(),
         "gpu_launches": calls,
-        "e2e": None,
-        "cpu_baseline": None,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
         "pages_context": "first 2 DiT blocks and first 12 denoising steps dense (Radial Attention, sec. 6)",
     }
     print(json.dumps(line), flush=True)
