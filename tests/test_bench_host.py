@@ -116,4 +116,7 @@ def test_traffic_record_key_tells_sink_masks_apart(bench):
     the plain mask of the same family."""
     assert bench.mask_key({"family": "radial"}) == "radial"
     assert bench.mask_key({"family": "radial", "sink_tokens": 3600}) == "radial+sink3600"
-    assert bench.recorded_traffic("hunyuan108k", "block", "radial+sink3600") is None
+    plain = bench.recorded_traffic("hunyuan108k", "block", "radial")
+    sink = bench.recorded_traffic("hunyuan108k", "block", "radial+sink3600")
+    assert sink is None or sink != plain
+    assert bench.recorded_traffic("hunyuan108k", "block", "radial+sink1") is None
