@@ -332,8 +332,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t ad = desc_add(q_desc, (kk >> 2) * L::Q_CHUNK_BYTES + (kk & 3) * 32);
                         const uint64_t bd = desc_add(kd, (kk >> 2) * L::H_CHUNK_BYTES + (kk & 3) * 32);
-                        if (leader)
-                            mma_ss(tmem + s_col_of(hh & 1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                        mma_ss(leader, tmem + s_col_of(hh & 1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                     }
                     if (leader) {
                         mma_commit(bar(B_S_FULL + (hh & 1)));
@@ -350,16 +349,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
 #pragma unroll
                     for (int kk = 0; kk < HALF / 16; ++kk) {
                         const uint64_t bd = desc_add(vd, kk * 2048);
-                        if (leader)
-                            mma_ts(tmem + O_COL, tmem + s_col_of(buf) + kk * 8, bd, idesc_pv,
-                                   (j > 0 || kk > 0) ? 1u : 0u);
+                        mma_ts(leader, tmem + O_COL, tmem + s_col_of(buf) + kk * 8, bd, idesc_pv,
+                               (j > 0 || kk > 0) ? 1u : 0u);
                     }
                     if (SPLIT_P) {
 #pragma unroll
                         for (int kk = 0; kk < HALF / 16; ++kk) {
                             const uint64_t bd = desc_add(vd, kk * 2048);
-                            if (leader)
-                                mma_ts(tmem + O_COL, tmem + s_col_of(buf) + HALF / 2 + kk * 8, bd, idesc_pv, 1u);
+                            mma_ts(leader, tmem + O_COL, tmem + s_col_of(buf) + HALF / 2 + kk * 8, bd, idesc_pv, 1u);
                         }
                     }
                     if (leader) {

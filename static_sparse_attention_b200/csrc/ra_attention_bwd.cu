@@ -301,8 +301,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
                     const uint64_t ad = desc_add(a, off), bd = desc_add(b2, off);
-                    if (leader)
-                        mma_ss(tmem + col, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    mma_ss(leader, tmem + col, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             // dQ += dS_j K_j: dS packed by the warpgroups, keys 16 kk .. 16 kk + 15
@@ -313,9 +312,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < TILE / 16; ++kk) {
                     const uint64_t bd = desc_add(kdesc, kk * 2048);
-                    if (leader)
-                        mma_ts(tmem + DQ_COL_ACC, tmem + dq_s_col(bf) + (kk >> 2) * 64 + (kk & 3) * 8, bd, idesc_acc,
-                               (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(leader, tmem + DQ_COL_ACC, tmem + dq_s_col(bf) + (kk >> 2) * 64 + (kk & 3) * 8, bd,
+                           idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 if (leader)
                     mma_commit(bar(BB::K_EMPTY + ks));
@@ -649,8 +647,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32;
                     const uint64_t ad = desc_add(a, off), bd = desc_add(b2, off);
-                    if (leader)
-                        mma_ss(tmem + col, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    mma_ss(leader, tmem + col, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             // dK += dS^T_j Q_j: dS^T packed by the warpgroups, queries 16 kk .. 16 kk + 15
@@ -664,9 +661,8 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                 for (int u = 0; u < 4; ++u) {
                     const int kk = 4 * (u >> 1) + 2 * half + (u & 1);
                     const uint64_t bd = desc_add(qdesc, kk * 2048);
-                    if (leader)
-                        mma_ts(tmem + KV_COL_DK, tmem + KV_COL_DP + (kk >> 2) * 64 + (kk & 3) * 8, bd, idesc_acc,
-                               (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(leader, tmem + KV_COL_DK, tmem + KV_COL_DP + (kk >> 2) * 64 + (kk & 3) * 8, bd,
+                           idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 if (leader && half == 1)
                     mma_commit(bar(BB::Q_EMPTY + qs));
@@ -679,8 +675,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                 for (int kk = 0; kk < TILE / 16; ++kk) {
                     const uint64_t ad = desc_add(dPTd, (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32);
                     const uint64_t bd = desc_add(odesc, kk * 2048);
-                    if (leader)
-                        mma_ss(tmem + KV_COL_DV, ad, bd, idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_ss(leader, tmem + KV_COL_DV, ad, bd, idesc_acc, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 if (leader) {
                     mma_commit(bar(BB::DV_DONE));
