@@ -582,7 +582,8 @@ def run_policy(args, c, mask, world, rank, dev):
     dense mask when t < dense_steps or l < dense_blocks, else the workload's
     sparse mask (the dense warm-up of the first steps and the dense first DiT
     blocks).  One timed step = one denoising step (policy_blocks calls); the
-    schedule runs policy_steps of them, so --steps / --warmup are not used."""
+    schedule runs policy_steps of them, so --steps is not used; --warmup (at
+    least 3) untimed calls of each mask precede the timed region."""
     import torch
     import torch.distributed as dist
 
@@ -607,10 +608,11 @@ def run_policy(args, c, mask, world, rank, dev):
     def call(m):
         ra.attention_fwd(q, k, v, m, scale=scale, mode=args.mode if m is sparse else "block", out=o, stream=stream)
 
-    # per-call times of each mask, for the all-dense and all-sparse reference points
+    # warm-up, and per-call times of each mask for the all-dense and all-sparse reference points
+    warmup = max(3, args.warmup)
     per_call = {}
     for name, m in (("sparse", sparse), ("dense", dense)):
-        for _ in range(2):
+        for _ in range(warmup):
             call(m)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -689,7 +691,7 @@ def run_policy(args, c, mask, world, rank, dev):
     achieved = flop / (total_ms / 1e3) / 1e12
     line = {
         "metric": METRIC_POLICY, "value": flop * world / (total_ms / 1e3) / 1e12, "unit": "TFLOP/s",
-        "n_gpus": world, "steps": T, "warmup": 2, "ms_per_step": total_ms / T, "higher_is_better": True,
+        "n_gpus": world, "steps": T, "warmup": warmup, "ms_per_step": total_ms / T, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {
             "workload": workload_desc(args.workload, mask, args.mode, c),
