@@ -39,7 +39,11 @@
 // dispatch order; identity when absent): query tiles sorted by in-frame
 // position band, then frame, so that the CTAs resident together share a
 // position band across many frames and walk overlapping key tiles of every
-// frame (eq. 4's bands are centred on the query's own in-frame position).
+// frame (eq. 4's bands are centred on the query's own in-frame position).  On
+// long sequences each CTA walks its row's key tiles of the frames near its own
+// first (the mask's walk: a contiguous segment of the ascending row), then the
+// others in ascending order, so that the resident CTAs stay closer together in
+// the far frames.
 //
 // Online softmax in base 2: x = S * scale * log2(e); p = 2^(x - m) with m a
 // running maximum that is only raised (and O, l rescaled) when a half-tile's
@@ -81,7 +85,7 @@ enum : int {
     SITE_Q_FULL = 1, SITE_K_EMPTY, SITE_V_EMPTY, SITE_K_FULL, SITE_P_FULL, SITE_V_FULL, SITE_S_FULL,
     SITE_PV_DONE, SITE_O_FINAL, SITE_SELFTEST, SITE_SMEM_ALIGN,
     // bounds checks of the debug build
-    SITE_B_QTILE = 40, SITE_B_ROW, SITE_B_KTILE, SITE_B_SELFTEST
+    SITE_B_QTILE = 40, SITE_B_ROW, SITE_B_KTILE, SITE_B_SELFTEST, SITE_B_WALK
 };
 
 template <int D>
@@ -125,6 +129,7 @@ struct FwdParams {
     const int* col_idx;
     const unsigned char* flag;
     const int* qorder; // query tile of CTA x (a permutation of [0, nb)), or null for x itself
+    const int* walk;   // [2 nb]: row offsets a, b of each row's near segment, walked first; or null
     int nnz;           // entries of col_idx / flag (bounds checks of the debug build)
     __nv_bfloat16* O;
     float* lse;
@@ -256,6 +261,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
     const int row_start = skip ? 0 : p.row_ptr[qb];
     const int L_row = skip ? 0 : p.row_ptr[qb + 1] - row_start;
     const int n_half = 2 * L_row;
+    // The order of the row's kept tiles: its near segment [wa, wb) first, then
+    // the others in ascending order (the identity without a walk).
+    int wa = 0, wb = 0;
+    if (p.walk && L_row > 0) {
+        wa = p.walk[2 * qb];
+        wb = p.walk[2 * qb + 1];
+        if (!in_bounds(wc, 0 <= wa && wa <= wb && wb <= L_row, SITE_B_WALK))  // (debug build)
+            wa = wb = 0;
+    }
+    auto walk = [wa, wb](int i) {
+        const int near = wb - wa;
+        return i < near ? wa + i : (i - near < wa ? i - near : i);
+    };
 
     if (warp == 4) {
         // ------------------------------------------------------------ producer
@@ -268,7 +286,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
                 tma_load_3d(sQ + c * L::Q_CHUNK_BYTES, &tmQ, bar(B_Q_FULL), c * 64, qb * TILE, bh);
             int k_issued = 0, v_issued = 0;
             for (int hh = 0; hh < n_half; ++hh) {
-                const int kb = p.col_idx[row_start + (hh >> 1)];
+                const int kb = p.col_idx[row_start + walk(hh >> 1)];
                 if (!in_bounds(wc, kb >= 0 && kb < p.nbk, SITE_B_KTILE))  // (debug build)
                     break;
                 const int key0 = kb * TILE + (hh & 1) * HALF;
@@ -383,8 +401,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
         uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
         bool masked = false;
         // CSR entry of the next tile, loaded one tile ahead of its use.
-        int next_kb = L_row > 0 ? p.col_idx[row_start] : 0;
-        int next_flag = L_row > 0 ? p.flag[row_start] : 0;
+        int next_kb = L_row > 0 ? p.col_idx[row_start + walk(0)] : 0;
+        int next_flag = L_row > 0 ? p.flag[row_start + walk(0)] : 0;
         for (int hh = 0; hh < n_half; ++hh) {
             const int i = hh >> 1, half = hh & 1, buf = hh & 1;
             const uint32_t s_col = s_col_of(buf);
@@ -394,8 +412,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
                 const int kb = next_kb;
                 const bool use_family = p.mode == RA_MODE_TOKEN_EXACT && next_flag != RA_TILE_FULL;
                 if (i + 1 < L_row) {
-                    next_kb = p.col_idx[row_start + i + 1];
-                    next_flag = p.flag[row_start + i + 1];
+                    next_kb = p.col_idx[row_start + walk(i + 1)];
+                    next_flag = p.flag[row_start + walk(i + 1)];
                 }
                 masked = use_family || (tail && kb == p.nbk - 1);
                 if (masked) {
@@ -679,6 +697,7 @@ extern "C" ra_status ra_attention_fwd(const void* Q, const void* K, const void* 
     p.col_idx = m->col_idx;
     p.flag = m->flag;
     p.qorder = m->qorder;
+    p.walk = m->walk;
     p.nnz = static_cast<int>(m->nnz);
     p.O = static_cast<__nv_bfloat16*>(O);
     p.lse = lse;

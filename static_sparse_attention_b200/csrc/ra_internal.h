@@ -28,6 +28,9 @@ struct ra_mask {
     // of the dQ pass runs query tile qorder[x], CTA x of the dK / dV pass key
     // tile qorder[x]; null when it is the identity.
     int* qorder;
+    // [2 nb]: the forward's walk of each CSR row (near frames first): row
+    // offsets a, b of the near segment; null when rows are walked in order.
+    int* walk;
 };
 
 namespace ra {

@@ -256,16 +256,17 @@ __global__ void __launch_bounds__(128) col_compact_kernel(const int* __restrict_
 // position band over many frames read overlapping key tiles; with the query
 // tiles of a head in plain order the resident CTAs instead cover a few whole
 // frames, i.e. every position, and at long sequences (a head's K and V well
-// beyond the L2 cache) re-read most key tiles from DRAM.  A band holds about
-// three query tiles per SM (1.5 times the forward's resident CTAs); masks of a
-// few such bands, and frames shorter than two tiles, keep the plain order.
-// Returns false when the order is the identity.
+// beyond the L2 cache) re-read most key tiles from DRAM.  The order is used from
+// about six query tiles per SM (three times the forward's resident CTAs) on, with
+// bands of about four query tiles per SM and at least two bands; smaller masks,
+// and frames shorter than two tiles, keep the plain order.  Returns false when
+// the order is the identity.
 bool dispatch_order(const MaskGeom& g, int nb, int sm_count, std::vector<int>& order)
 {
-    const long long per_band = 3LL * (sm_count > 0 ? sm_count : 148);
-    const int bands = static_cast<int>((nb + per_band / 2) / per_band);
-    if (g.s < 2 * TILE || bands < 2)
+    const long long sms = sm_count > 0 ? sm_count : 148;
+    if (g.s < 2 * TILE || (nb + 3 * sms / 2) / (3 * sms) < 2)
         return false;
+    const int bands = static_cast<int>(std::max<long long>(2, (nb + 2 * sms) / (4 * sms)));
     order.resize(nb);
     for (int q = 0; q < nb; ++q)
         order[q] = q;
@@ -278,6 +279,54 @@ bool dispatch_order(const MaskGeom& g, int nb, int sm_count, std::vector<int>& o
     return true;
 }
 
+// The forward kernel's walk of each query tile's CSR row, for long radial
+// masks (used with the dispatch order above): first the key tiles of the frames near
+// the query tile's own (those whose first row lies in a frame less than `near`
+// frames from the frame of the query tile's first row: a contiguous segment
+// [a, b) of the ascending row), then the others in ascending order.  The CTAs
+// resident together (one position band over consecutive frames) then take
+// their near frames, where a row spends most of its tiles, at about the same
+// time, and afterwards the far frames, where eq. 4 keeps a few tiles around the
+// band's positions, in the same ascending order.  (A mask that keeps whole far
+// frames, such as the dense one, would only stagger the CTAs' starting frames.)
+// walk[2 q], walk[2 q + 1] = a, b as offsets in the row.
+__global__ void __launch_bounds__(128) walk_kernel(MaskGeom g, int nb, int near, const int* __restrict__ row_ptr,
+                                                   const int* __restrict__ col_idx, int* __restrict__ walk)
+{
+    const int q = blockIdx.x * blockDim.x + threadIdx.x;
+    if (q >= nb)
+        return;
+    const long long i = static_cast<long long>(q) * TILE / g.s;  // frame of the tile's first row
+    const long long f_lo = i - near + 1, f_hi = i + near - 1;
+    // first key tile whose first row lies in frame >= f_lo; last one in frame <= f_hi
+    const long long k_lo = f_lo <= 0 ? 0 : (f_lo * g.s + TILE - 1) / TILE;
+    const long long k_hi = ((f_hi + 1) * g.s - 1) / TILE;
+    const int start = row_ptr[q], end = row_ptr[q + 1];
+    int lo = start, hi = end;
+    while (lo < hi) {  // lower bound of k_lo
+        const int mid = (lo + hi) >> 1;
+        if (col_idx[mid] < k_lo)
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    const int a = lo;
+    hi = end;
+    while (lo < hi) {  // upper bound of k_hi
+        const int mid = (lo + hi) >> 1;
+        if (col_idx[mid] <= k_hi)
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    walk[2 * q] = a - start;
+    walk[2 * q + 1] = lo - start;
+}
+
+// Frames from which the forward walks a radial mask's near frames first, and their reach.
+constexpr int WALK_MIN_FRAMES = 64;
+inline int walk_near_frames(const MaskGeom& g) { return g.f / 4; }
+
 void free_mask_arrays(ra_mask* m)
 {
     cudaFree(m->row_ptr);
@@ -288,7 +337,8 @@ void free_mask_arrays(ra_mask* m)
     cudaFree(m->row_idx);
     cudaFree(m->tflag);
     cudaFree(m->qorder);
-    m->row_ptr = m->col_idx = m->count = m->col_ptr = m->row_idx = m->qorder = nullptr;
+    cudaFree(m->walk);
+    m->row_ptr = m->col_idx = m->count = m->col_ptr = m->row_idx = m->qorder = m->walk = nullptr;
     m->flag = m->tflag = nullptr;
 }
 
@@ -446,6 +496,14 @@ extern "C" ra_status ra_build_mask(int family, int f, int s, const ra_mask_param
         // synchronous copy from pageable memory: `order` is released on return
         if ((e = cudaMemcpy(m->qorder, order.data(), sizeof(int) * nb, cudaMemcpyHostToDevice)) != cudaSuccess)
             return bail(e, "qorder copy");
+        if (nnz > 0 && g.family == FAM_RADIAL && g.f >= WALK_MIN_FRAMES) {
+            if ((e = cudaMalloc(&m->walk, sizeof(int) * 2 * static_cast<size_t>(nb))) != cudaSuccess)
+                return bail(e, "walk");
+            walk_kernel<<<(nb + 127) / 128, 128, 0, cs>>>(g, nb, walk_near_frames(g), m->row_ptr, m->col_idx,
+                                                           m->walk);
+            if ((e = cudaGetLastError()) != cudaSuccess)
+                return bail(e, "walk_kernel launch");
+        }
     }
     // The scratch arrays are released by ~Scratch; cudaFree waits for the kernels.
     if ((e = cudaStreamSynchronize(cs)) != cudaSuccess)

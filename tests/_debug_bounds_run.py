@@ -54,6 +54,17 @@ def main():
             _gpu.assert_close(_gpu.gather_rows(_gpu.to_f64(o), rows_bh, rows_q), want, f"debug {spec} {mode}")
             for g in grads:
                 assert bool(torch.isfinite(g).all()), f"debug {spec} {mode}: non-finite gradient"
+    # a radial mask long enough for the forward's near-first row walk (its row
+    # offsets are checked too), on seeded rows
+    spec, B, H, d = oracle.MaskSpec(oracle.RADIAL, 64, 1408), 1, 1, 128
+    Qh, Kh, Vh = (synth.normal_bf16(5300, t, (B, H, spec.n, d)) for t in range(3))
+    q, k, v = (_gpu.to_device(t) for t in (Qh, Kh, Vh))
+    m = ra.Mask("radial", spec.f, spec.s)
+    o = ra.attention_fwd(q, k, v, m, scale=1.0 / math.sqrt(d), mode="block")
+    status(f"{spec} walk")
+    rows_bh, rows_q = _gpu.sampled_rows(5300, spec.f, spec.s, B, H, 256)
+    want, _, _ = orc.attention_rows(Qh, Kh, Vh, spec, oracle.BLOCK, 1.0 / math.sqrt(d), rows_bh, rows_q)
+    _gpu.assert_close(_gpu.gather_rows(_gpu.to_f64(o), rows_bh, rows_q), want, f"debug {spec} walk")
     # the streaming SWC step (the forward over the ring with its own tile lists)
     s, W, B, H, d = 130, 3, 1, 2, 128
     Qh, Kh, Vh = (synth.normal_bf16(5200, t, (B, H, 6 * s, d)) for t in range(3))

@@ -194,6 +194,23 @@ def test_bounded_wait_selftest_reports_timeout():
     assert float(x.sum()) == 4.0
 
 
+# ------------------------------------------ near-first row walk (sampled rows)
+
+# A radial mask long enough for the forward's near-first walk of each CSR row
+# (at least 64 frames, with the position-band dispatch order: about six query
+# tiles per SM): 64 frames of 1408 tokens, 704 query tiles.
+WALK_SPEC = oracle.MaskSpec(oracle.RADIAL, 64, 1408)
+
+
+@pytest.mark.parametrize("mode", ["block", "token_exact"])
+def test_near_first_walk_sampled_rows(orc, mode):
+    _gpu.need_gpu()
+    B, H, d = 1, 2, 128
+    Q, K, V = (synth.normal_bf16(6400, t, (B, H, WALK_SPEC.n, d)) for t in range(3))
+    rows = _gpu.sampled_rows(6400, WALK_SPEC.f, WALK_SPEC.s, B, H, 256)
+    _check(orc, WALK_SPEC, Q, K, V, mode, rows=rows, what=f"near-first walk {mode}")
+
+
 # ------------------------------------------------- full-size configs (sampled)
 
 FULL = [("wan_radial", 0, "block"), ("wan_radial", 1, "block"), ("hunyuan108k", 0, "block"),
