@@ -249,6 +249,11 @@ __global__ void __launch_bounds__(128) col_compact_kernel(const int* __restrict_
     }
 }
 
+// Frames from which the forward walks a radial mask's near frames first, and their reach.
+constexpr int WALK_MIN_FRAMES = 64;
+inline int walk_near_frames(const MaskGeom& g) { return g.f / 4; }
+inline bool walked(const MaskGeom& g) { return g.family == FAM_RADIAL && g.f >= WALK_MIN_FRAMES; }
+
 // The order in which the attention kernels' CTAs take their tiles (query tiles
 // of the forward and the dQ pass, key tiles of the dK / dV pass, by the mask's
 // symmetry in query and key): sorted by in-frame position band, then by frame.  eq. 4 keeps, in every key frame, a band of
@@ -258,15 +263,17 @@ __global__ void __launch_bounds__(128) col_compact_kernel(const int* __restrict_
 // frames, i.e. every position, and at long sequences (a head's K and V well
 // beyond the L2 cache) re-read most key tiles from DRAM.  The order is used from
 // about six query tiles per SM (three times the forward's resident CTAs) on, with
-// bands of about four query tiles per SM and at least two bands; smaller masks,
-// and frames shorter than two tiles, keep the plain order.  Returns false when
-// the order is the identity.
-bool dispatch_order(const MaskGeom& g, int nb, int sm_count, std::vector<int>& order)
+// bands of about three query tiles per SM, or four for the masks whose rows the
+// forward walks near frames first (walk_kernel below; measured with that walk),
+// and at least two bands; smaller masks, and frames shorter than two tiles, keep
+// the plain order.  Returns false when the order is the identity.
+bool dispatch_order(const MaskGeom& g, int nb, int sm_count, bool walk_rows, std::vector<int>& order)
 {
     const long long sms = sm_count > 0 ? sm_count : 148;
     if (g.s < 2 * TILE || (nb + 3 * sms / 2) / (3 * sms) < 2)
         return false;
-    const int bands = static_cast<int>(std::max<long long>(2, (nb + 2 * sms) / (4 * sms)));
+    const long long per_band = (walk_rows ? 4 : 3) * sms;
+    const int bands = static_cast<int>(std::max<long long>(2, (nb + per_band / 2) / per_band));
     order.resize(nb);
     for (int q = 0; q < nb; ++q)
         order[q] = q;
@@ -323,9 +330,6 @@ __global__ void __launch_bounds__(128) walk_kernel(MaskGeom g, int nb, int near,
     walk[2 * q + 1] = lo - start;
 }
 
-// Frames from which the forward walks a radial mask's near frames first, and their reach.
-constexpr int WALK_MIN_FRAMES = 64;
-inline int walk_near_frames(const MaskGeom& g) { return g.f / 4; }
 
 void free_mask_arrays(ra_mask* m)
 {
@@ -490,13 +494,13 @@ extern "C" ra_status ra_build_mask(int family, int f, int s, const ra_mask_param
     if ((e = cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, device)) != cudaSuccess)
         return bail(e, "SM count");
     std::vector<int> order;
-    if (dispatch_order(g, nb, sm_count, order)) {
+    if (dispatch_order(g, nb, sm_count, walked(g), order)) {
         if ((e = cudaMalloc(&m->qorder, sizeof(int) * nb)) != cudaSuccess)
             return bail(e, "qorder");
         // synchronous copy from pageable memory: `order` is released on return
         if ((e = cudaMemcpy(m->qorder, order.data(), sizeof(int) * nb, cudaMemcpyHostToDevice)) != cudaSuccess)
             return bail(e, "qorder copy");
-        if (nnz > 0 && g.family == FAM_RADIAL && g.f >= WALK_MIN_FRAMES) {
+        if (nnz > 0 && walked(g)) {
             if ((e = cudaMalloc(&m->walk, sizeof(int) * 2 * static_cast<size_t>(nb))) != cudaSuccess)
                 return bail(e, "walk");
             walk_kernel<<<(nb + 127) / 128, 128, 0, cs>>>(g, nb, walk_near_frames(g), m->row_ptr, m->col_idx,
