@@ -262,7 +262,7 @@ inline bool walked(const MaskGeom& g) { return g.family == FAM_RADIAL && g.f >= 
 // tiles of a head in plain order the resident CTAs instead cover a few whole
 // frames, i.e. every position, and at long sequences (a head's K and V well
 // beyond the L2 cache) re-read most key tiles from DRAM.  The order is used from
-// about six query tiles per SM (three times the forward's resident CTAs) on, with
+// about 4.5 query tiles per SM (2.25 times the forward's resident CTAs) on, with
 // bands of about three query tiles per SM, or four for the masks whose rows the
 // forward walks near frames first (walk_kernel below; measured with that walk),
 // and at least two bands; smaller masks, and frames shorter than two tiles, keep
@@ -329,7 +329,6 @@ __global__ void __launch_bounds__(128) walk_kernel(MaskGeom g, int nb, int near,
     walk[2 * q] = a - start;
     walk[2 * q + 1] = lo - start;
 }
-
 
 void free_mask_arrays(ra_mask* m)
 {
