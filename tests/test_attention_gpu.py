@@ -197,8 +197,8 @@ def test_bounded_wait_selftest_reports_timeout():
 # ------------------------------------------ near-first row walk (sampled rows)
 
 # A radial mask long enough for the forward's near-first walk of each CSR row
-# (at least 64 frames, with the position-band dispatch order: about six query
-# tiles per SM): 64 frames of 1408 tokens, 704 query tiles.
+# (at least 64 frames, with the position-band dispatch order: from about 4.5
+# query tiles per SM, 666 on 148 SMs): 64 frames of 1408 tokens, 704 query tiles.
 WALK_SPEC = oracle.MaskSpec(oracle.RADIAL, 64, 1408)
 
 
