@@ -39,7 +39,31 @@ constexpr float LOG2E = 1.4426950408889634f;
 enum : int { BSITE_RES = 21, BSITE_X_EMPTY, BSITE_Y_EMPTY, BSITE_X_FULL, BSITE_Y_FULL, BSITE_S_FULL, BSITE_DS_FULL,
              BSITE_ACC, BSITE_FINAL,
              // bounds checks of the debug build
-             BSITE_B_ROW = 50, BSITE_B_TILE };
+             BSITE_B_ROW = 50, BSITE_B_TILE, BSITE_B_WALK };
+
+// The order in which a CTA takes the entries of its CSR row: the row's near
+// segment [a, b) first, then the others in ascending order (the identity
+// without a walk array).
+struct RowWalk {
+    int a = 0, b = 0;
+    __device__ int operator()(int i) const
+    {
+        const int near = b - a;
+        return i < near ? a + i : (i - near < a ? i - near : i);
+    }
+};
+
+__device__ __forceinline__ RowWalk row_walk(const int* walk, int tile, int len, const WaitCtl& wc)
+{
+    RowWalk w;
+    if (walk && len > 0) {
+        w.a = walk[2 * tile];
+        w.b = walk[2 * tile + 1];
+        if (!in_bounds(wc, 0 <= w.a && w.a <= w.b && w.b <= len, BSITE_B_WALK))  // (debug build)
+            w.a = w.b = 0;
+    }
+    return w;
+}
 
 struct BwdParams {
     MaskGeom g;
@@ -48,6 +72,7 @@ struct BwdParams {
     const int* idx;            // col_idx or row_idx
     const unsigned char* flag; // flag or tflag
     const int* order;          // tile of CTA x (the mask's dispatch order), or null for x itself
+    const int* walk;           // [2 nb]: offsets a, b of each row's near segment, walked first; or null
     int nnz;                   // entries of idx / flag (bounds checks of the debug build)
     const float* lse;          // [B*H, n] natural log
     const float* Dv;           // [B*H, n] rowsum(dO * O)
@@ -245,6 +270,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
     const bool skip = *abort_flag != 0;
     const int start = skip ? 0 : p.ptr[qb];
     const int len = skip ? 0 : p.ptr[qb + 1] - start;
+    const RowWalk walk = row_walk(p.walk, qb, len, wc);
 
     if (warp == DQ_PRODUCER_WARP) {
         // ------------------------------------------------------------ producer
@@ -256,7 +282,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
             }
             int k_issued = 0, v_issued = 0;
             for (int j = 0; j < len; ++j) {
-                const int tile = p.idx[start + j];
+                const int tile = p.idx[start + walk(j)];
                 if (!in_bounds(wc, tile >= 0 && tile < p.nb, BSITE_B_TILE))  // (debug build)
                     break;
                 const int row0 = tile * TILE;
@@ -381,15 +407,15 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
         const uint64_t c2 = f2pack(p.scale_log2, p.scale_log2), nl2 = f2pack(nl, nl), nd2 = f2pack(-row_d, -row_d);
         bool ok = true;
         // CSR entry of the next step, loaded one step ahead of its use
-        int next_kb = len > 0 ? p.idx[start] : 0;
-        int next_flag = len > 0 ? p.flag[start] : 0;
+        int next_kb = len > 0 ? p.idx[start + walk(0)] : 0;
+        int next_flag = len > 0 ? p.flag[start + walk(0)] : 0;
         for (int j = 0; j < len; ++j) {
             const int bf = j & 1;
             const int kb = next_kb;
             const bool use_family = p.mode == RA_MODE_TOKEN_EXACT && next_flag != RA_TILE_FULL;
             if (j + 1 < len) {
-                next_kb = p.idx[start + j + 1];
-                next_flag = p.flag[start + j + 1];
+                next_kb = p.idx[start + walk(j + 1)];
+                next_flag = p.flag[start + walk(j + 1)];
             }
             const bool masked = use_family || (tail && kb == p.nb - 1);
             uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
@@ -589,6 +615,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
     const bool skip = *abort_flag != 0;
     const int start = skip ? 0 : p.ptr[kb];
     const int len = skip ? 0 : p.ptr[kb + 1] - start;
+    const RowWalk walk = row_walk(p.walk, kb, len, wc);
 
     if (warp == KV_PRODUCER_WARP) {
         // ------------------------------------------------------------ producer
@@ -600,7 +627,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
             }
             int q_issued = 0, o_issued = 0;
             for (int j = 0; j < len; ++j) {
-                const int tile = p.idx[start + j];
+                const int tile = p.idx[start + walk(j)];
                 if (!in_bounds(wc, tile >= 0 && tile < p.nb, BSITE_B_TILE))  // (debug build)
                     break;
                 const int row0 = tile * TILE;
@@ -765,16 +792,16 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
             return l > -INFINITY ? -(l * LOG2E) : -INFINITY;
         };
         const uint64_t c2 = f2pack(p.scale_log2, p.scale_log2);
-        int next_qb = len > 0 ? p.idx[start] : 0;
-        int next_flag = len > 0 ? p.flag[start] : 0;
+        int next_qb = len > 0 ? p.idx[start + walk(0)] : 0;
+        int next_flag = len > 0 ? p.flag[start + walk(0)] : 0;
         float next_stat = len > 0 ? column_stat(next_qb) : 0.f;
         for (int j = 0; j < len; ++j) {
             const int qb = next_qb;
             const bool masked = p.mode == RA_MODE_TOKEN_EXACT && next_flag != RA_TILE_FULL;
             const float stat = next_stat;
             if (j + 1 < len) {
-                next_qb = p.idx[start + j + 1];
-                next_flag = p.flag[start + j + 1];
+                next_qb = p.idx[start + walk(j + 1)];
+                next_flag = p.flag[start + walk(j + 1)];
                 next_stat = column_stat(next_qb);
             }
             // keep bits of this warpgroup's two 32-column chunks
@@ -993,6 +1020,7 @@ ra_status run_bwd(const void* Q, const void* K, const void* V, const void* O, co
     p.ptr = m->row_ptr;
     p.idx = m->col_idx;
     p.flag = m->flag;
+    p.walk = m->walk;
     p.out0 = static_cast<__nv_bfloat16*>(dQ);
     p.out1 = nullptr;
     if ((st = launch_dq<D>(rq, rdo, rk, rv, p, B, cs)) != RA_OK)
@@ -1001,6 +1029,7 @@ ra_status run_bwd(const void* Q, const void* K, const void* V, const void* O, co
     p.ptr = m->col_ptr;
     p.idx = m->row_idx;
     p.flag = m->tflag;
+    p.walk = m->walk_t;
     p.out0 = static_cast<__nv_bfloat16*>(dK);
     p.out1 = static_cast<__nv_bfloat16*>(dV);
     return launch_dkdv<D>(rk, rv, rq, rdo, p, B, cs);

@@ -28,9 +28,11 @@ struct ra_mask {
     // of the dQ pass runs query tile qorder[x], CTA x of the dK / dV pass key
     // tile qorder[x]; null when it is the identity.
     int* qorder;
-    // [2 nb]: the forward's walk of each CSR row (near frames first): row
-    // offsets a, b of the near segment; null when rows are walked in order.
+    // [2 nb]: the walk of each CSR row (near frames first) by the forward and
+    // the dQ pass: row offsets a, b of the near segment; null when rows are
+    // walked in order.  walk_t: the same for the transposed CSR (dK / dV pass).
     int* walk;
+    int* walk_t;
 };
 
 namespace ra {

@@ -341,7 +341,8 @@ void free_mask_arrays(ra_mask* m)
     cudaFree(m->tflag);
     cudaFree(m->qorder);
     cudaFree(m->walk);
-    m->row_ptr = m->col_idx = m->count = m->col_ptr = m->row_idx = m->qorder = m->walk = nullptr;
+    cudaFree(m->walk_t);
+    m->row_ptr = m->col_idx = m->count = m->col_ptr = m->row_idx = m->qorder = m->walk = m->walk_t = nullptr;
     m->flag = m->tflag = nullptr;
 }
 
@@ -506,6 +507,14 @@ extern "C" ra_status ra_build_mask(int family, int f, int s, const ra_mask_param
                                                            m->walk);
             if ((e = cudaGetLastError()) != cudaSuccess)
                 return bail(e, "walk_kernel launch");
+            // the transposed CSR's rows (key tiles, their query tiles): the same
+            // walk, by the mask's symmetry in query and key
+            if ((e = cudaMalloc(&m->walk_t, sizeof(int) * 2 * static_cast<size_t>(nb))) != cudaSuccess)
+                return bail(e, "walk_t");
+            walk_kernel<<<(nb + 127) / 128, 128, 0, cs>>>(g, nb, walk_near_frames(g), m->col_ptr, m->row_idx,
+                                                           m->walk_t);
+            if ((e = cudaGetLastError()) != cudaSuccess)
+                return bail(e, "walk_kernel launch (transposed)");
         }
     }
     // The scratch arrays are released by ~Scratch; cudaFree waits for the kernels.

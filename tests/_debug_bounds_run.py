@@ -60,8 +60,12 @@ def main():
     Qh, Kh, Vh = (synth.normal_bf16(5300, t, (B, H, spec.n, d)) for t in range(3))
     q, k, v = (_gpu.to_device(t) for t in (Qh, Kh, Vh))
     m = ra.Mask("radial", spec.f, spec.s)
-    o = ra.attention_fwd(q, k, v, m, scale=1.0 / math.sqrt(d), mode="block")
+    lse = torch.empty((B, H, spec.n), dtype=torch.float32, device="cuda")
+    o = ra.attention_fwd(q, k, v, m, scale=1.0 / math.sqrt(d), mode="block", lse=lse)
+    grads = ra.attention_bwd(q, k, v, o, torch.randn_like(o), lse, m, scale=1.0 / math.sqrt(d), mode="block")
     status(f"{spec} walk")
+    for g in grads:
+        assert bool(torch.isfinite(g).all()), f"debug {spec} walk: non-finite gradient"
     rows_bh, rows_q = _gpu.sampled_rows(5300, spec.f, spec.s, B, H, 256)
     want, _, _ = orc.attention_rows(Qh, Kh, Vh, spec, oracle.BLOCK, 1.0 / math.sqrt(d), rows_bh, rows_q)
     _gpu.assert_close(_gpu.gather_rows(_gpu.to_f64(o), rows_bh, rows_q), want, f"debug {spec} walk")

@@ -249,3 +249,26 @@ def test_wan_sampled_key_rows(orc):
     c = synth.CONFIGS["wan_radial"]
     keys = synth.sample_rows(synth.config_seed("wan_radial") + 1, c["f"], c["s"], 24)
     _key_rows_check(orc, "wan_radial", 0, 1, keys, "wan")
+
+
+@pytest.mark.parametrize("mode", ["block", "token_exact"])
+def test_near_first_walk_backward_sampled_rows(orc, mode):
+    """A radial mask long enough for the near-first walk of the rows of both the
+    block-CSR (dQ pass) and its transpose (dK / dV pass): 64 frames of 1408
+    tokens, 704 tiles.  dQ on 256 seeded query rows and dK, dV on the 6 boundary
+    key rows (first and last of the sequence, of frame 1 and of the last frame,
+    first of the last tile) against the oracle."""
+    _gpu.need_gpu()
+    spec = oracle.MaskSpec(oracle.RADIAL, 64, 1408)
+    B, H, d = 1, 1, 128
+    Qh, Kh, Vh, dOh = (synth.normal_bf16(6500, t, (B, H, spec.n, d)) for t in (0, 1, 2, synth.DOUT_TENSOR_ID))
+    dq, dk, dv, _ = _fwd_bwd(spec, Qh, Kh, Vh, dOh, mode)
+    scale = _gpu.scale_for(d)
+    row_bh, row_q = _gpu.sampled_rows(6500, spec.f, spec.s, B, H, count=256)
+    want = orc.attention_bwd_query_rows(Qh, Kh, Vh, dOh, spec, MODES[mode], scale, row_bh, row_q)
+    assert_grad_close(_gpu.gather_rows(_gpu.to_f64(dq), row_bh, row_q), want, f"walk {mode} dQ sampled")
+    keys = synth.sample_rows(6501, spec.f, spec.s, 4)  # the boundary rows
+    want_k, want_v = orc.attention_bwd_key_rows(Qh[0, 0], Kh[0, 0], Vh[0, 0], dOh[0, 0], spec, MODES[mode], scale,
+                                                keys)
+    assert_grad_close(_gpu.to_f64(dk)[0, 0, keys], want_k, f"walk {mode} dK sampled")
+    assert_grad_close(_gpu.to_f64(dv)[0, 0, keys], want_v, f"walk {mode} dV sampled")
