@@ -286,8 +286,10 @@ bool dispatch_order(const MaskGeom& g, int nb, int sm_count, bool walk_rows, std
     return true;
 }
 
-// The forward kernel's walk of each query tile's CSR row, for long radial
-// masks (used with the dispatch order above): first the key tiles of the frames near
+// The walk of each query tile's CSR row by the forward and the dQ pass (and,
+// computed over the transposed CSR, of each key tile's row by the dK / dV pass,
+// by the mask's symmetry), for long radial masks (used with the dispatch order
+// above): first the key tiles of the frames near
 // the query tile's own (those whose first row lies in a frame less than `near`
 // frames from the frame of the query tile's first row: a contiguous segment
 // [a, b) of the ascending row), then the others in ascending order.  The CTAs
